@@ -1,0 +1,288 @@
+"""Pins of the fp64 oracle to facts fixed outside the oracle itself.
+
+Each test would fail on a plausible slip in ``oracle/`` (a dropped term, a
+wrong sign or index, a transposed operand, a wrong GQA mapping or mask):
+closed-form worked examples (tests/golden), invariants of the definition of
+exact attention, brute force on tiny inputs, finite differences of the
+forward, an independent library routine (torch's fp64 CPU scaled dot-product
+attention and autograd), and the tiled online-softmax algorithm.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.attention import attention_head
+import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "closed_form.json")
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# --- closed forms -----------------------------------------------------------
+
+def test_golden_closed_forms():
+    cases = json.load(open(GOLD))["cases"]
+    for c in cases:
+        q, k, v = (np.array(c[n])[None, :, None, :] for n in ("q", "k", "v"))
+        O, L = oracle.attn_fwd(q, k, v, c["causal"], c["scale"])
+        np.testing.assert_allclose(O[0, :, 0], np.array(c["o"]), rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L[0, 0], np.array(c["lse"]), rtol=0, atol=1e-13)
+        if "do" in c:
+            do = np.array(c["do"])[None, :, None, :]
+            dq, dk, dv = oracle.attn_bwd(q, k, v, do, c["causal"], c["scale"])
+            np.testing.assert_allclose(dq[0, :, 0], np.array(c["dq"]), atol=1e-13)
+            np.testing.assert_allclose(dk[0, :, 0], np.array(c["dk"]), atol=1e-13)
+            np.testing.assert_allclose(dv[0, :, 0], np.array(c["dv"]), atol=1e-13)
+
+
+# --- invariants (C4 - C6f) --------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_sum_to_one(causal):
+    q, k, v = _rand((37, 8), 1), _rand((37, 8), 2), _rand((37, 8), 3)
+    _, lse, P = attention_head(q, k, v, causal, 0.3)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, atol=1e-12)
+    if causal:
+        assert np.all(np.triu(P, 1) == 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_v_all_ones_gives_ones(causal):
+    q, k = _rand((2, 50, 3, 16), 4), _rand((2, 50, 3, 16), 5)
+    v = np.ones((2, 50, 3, 16))
+    O, _ = oracle.attn_fwd(q, k, v, causal, 0.25)
+    assert np.max(np.abs(O - 1.0)) <= 1e-14
+    dq, dk, dv = oracle.attn_bwd(q, k, v, _rand((2, 50, 3, 16), 6), causal, 0.25)
+    assert np.max(np.abs(dq)) < 1e-12 and np.max(np.abs(dk)) < 1e-12
+
+
+def test_causal_row0_is_v0():
+    q, k, v = _rand((1, 40, 2, 8), 7), _rand((1, 40, 2, 8), 8), _rand((1, 40, 2, 8), 9)
+    O, L = oracle.attn_fwd(q, k, v, True, 0.7)
+    np.testing.assert_allclose(O[:, 0], v[:, 0], atol=1e-14)
+    np.testing.assert_allclose(L[0, :, 0], 0.7 * np.einsum("hd,hd->h", q[0, 0], k[0, 0]), atol=1e-13)
+
+
+def test_single_key():
+    q, k, v = _rand((3, 1, 2, 8), 10), _rand((3, 1, 2, 8), 11), _rand((3, 1, 2, 8), 12)
+    for causal in (False, True):
+        O, L = oracle.attn_fwd(q, k, v, causal, 0.5)
+        np.testing.assert_allclose(O, v, atol=1e-14)
+        np.testing.assert_allclose(L, 0.5 * np.einsum("bnhd,bnhd->bhn", q, k), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_is_uniform(causal):
+    N = 33
+    q = np.zeros((1, N, 1, 4))
+    k, v = _rand((1, N, 1, 4), 13), _rand((1, N, 1, 4), 14)
+    O, L = oracle.attn_fwd(q, k, v, causal, 1.0)
+    if causal:
+        want = np.cumsum(v[0, :, 0], axis=0) / np.arange(1, N + 1)[:, None]
+        lse = np.log(np.arange(1, N + 1))
+    else:
+        want = np.broadcast_to(v[0, :, 0].mean(axis=0), (N, 4))
+        lse = np.full(N, np.log(N))
+    np.testing.assert_allclose(O[0, :, 0], want, atol=1e-13)
+    np.testing.assert_allclose(L[0, 0], lse, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_shift(causal):
+    q, k, v = _rand((1, 30, 1, 6), 15), _rand((1, 30, 1, 6), 16), _rand((1, 30, 1, 6), 17)
+    u = _rand((6,), 18)
+    O1, L1 = oracle.attn_fwd(q, k, v, causal, 0.4)
+    O2, L2 = oracle.attn_fwd(q, k + u, v, causal, 0.4)
+    np.testing.assert_allclose(O2, O1, atol=1e-12)
+    np.testing.assert_allclose(L2[0, 0], L1[0, 0] + 0.4 * q[0, :, 0] @ u, atol=1e-12)
+
+
+def test_kv_permutation_noncausal():
+    q, k, v = _rand((1, 25, 2, 6), 19), _rand((1, 25, 2, 6), 20), _rand((1, 25, 2, 6), 21)
+    perm = np.random.default_rng(22).permutation(25)
+    O1, L1 = oracle.attn_fwd(q, k, v, False, 0.4)
+    O2, L2 = oracle.attn_fwd(q, k[:, perm], v[:, perm], False, 0.4)
+    np.testing.assert_allclose(O2, O1, atol=1e-13)
+    np.testing.assert_allclose(L2, L1, atol=1e-13)
+
+
+def test_bwd_equal_keys_zero_dq():
+    q, v, do = _rand((1, 12, 1, 5), 23), _rand((1, 12, 1, 5), 24), _rand((1, 12, 1, 5), 25)
+    k = np.broadcast_to(_rand((5,), 26), (1, 12, 1, 5)).copy()
+    dq, _, _ = oracle.attn_bwd(q, k, v, do, False, 0.9)
+    assert np.max(np.abs(dq)) < 1e-12
+
+
+# --- brute force and an independent library routine ------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_loops(causal):
+    """Pure-Python triple loop on a tiny case (no matmul, no vectorised softmax)."""
+    N, d, scale = 5, 3, 0.8
+    q, k, v = _rand((N, d), 27), _rand((N, d), 28), _rand((N, d), 29)
+    O, L, _ = attention_head(q, k, v, causal, scale)
+    import math
+    for i in range(N):
+        keys = [j for j in range(N) if not (causal and j > i)]
+        s = [scale * sum(q[i, c] * k[j, c] for c in range(d)) for j in keys]
+        den = sum(math.exp(x) for x in s)
+        for c in range(d):
+            assert abs(O[i, c] - sum(math.exp(x) * v[j, c] for x, j in zip(s, keys)) / den) < 1e-13
+        assert abs(L[i] - math.log(den)) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_matches_torch_sdpa_fp64(causal):
+    B, N, Hq, Hkv, d, scale = 2, 70, 4, 2, 16, 0.3
+    q, k, v = _rand((B, N, Hq, d), 30), _rand((B, N, Hkv, d), 31), _rand((B, N, Hkv, d), 32)
+    do = _rand((B, N, Hq, d), 33)
+    O, L = oracle.attn_fwd(q, k, v, causal, scale)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, causal, scale)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64).transpose(1, 2).requires_grad_() for x in (q, k, v))
+    rep = Hq // Hkv
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(rep, dim=1), tv.repeat_interleave(rep, dim=1), is_causal=causal, scale=scale)
+    np.testing.assert_allclose(O, to.detach().transpose(1, 2).numpy(), atol=1e-12)
+    to.backward(torch.tensor(do).transpose(1, 2))
+    np.testing.assert_allclose(dq, tq.grad.transpose(1, 2).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.transpose(1, 2).numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.transpose(1, 2).numpy(), atol=1e-11)
+    # LSE pinned by torch's logsumexp of the scaled, masked scores
+    s = scale * torch.einsum("bhnd,bhmd->bhnm", tq.detach(), tk.detach().repeat_interleave(rep, dim=1))
+    if causal:
+        s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+    np.testing.assert_allclose(L, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
+
+
+# --- finite differences (C8) -------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_finite_differences(causal):
+    B, N, H, d, scale = 1, 8, 1, 4, 0.6
+    q, k, v = _rand((B, N, H, d), 34), _rand((B, N, H, d), 35), _rand((B, N, H, d), 36)
+    W = _rand((B, N, H, d), 37)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, W, causal, scale)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(oracle.attn_fwd(q_, k_, v_, causal, scale)[0] * W))
+
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (loss(**{a + "_": b for a, b in args_p.items()}) -
+                        loss(**{a + "_": b for a, b in args_m.items()})) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8)
+
+
+# --- structure: GQA, varlen, sampled rows, merge (C8b, C8c, C10) ------------
+
+def test_gqa_equals_repeated_mha():
+    B, N, Hq, Hkv, d = 1, 20, 6, 2, 8
+    q, k, v, do = (_rand((B, N, h, d), s) for h, s in ((Hq, 38), (Hkv, 39), (Hkv, 40), (Hq, 41)))
+    O, L = oracle.attn_fwd(q, k, v, True, 0.35)
+    kr, vr = np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2)
+    O2, L2 = oracle.attn_fwd(q, kr, vr, True, 0.35)
+    np.testing.assert_allclose(O, O2, atol=1e-14)
+    np.testing.assert_allclose(L, L2, atol=1e-14)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, True, 0.35)
+    dq2, dk2, dv2 = oracle.attn_bwd(q, kr, vr, do, True, 0.35)
+    np.testing.assert_allclose(dq, dq2, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(B, N, Hkv, 3, d).sum(axis=3), atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, N, Hkv, 3, d).sum(axis=3), atol=1e-13)
+    # contiguous groups: query head 1 reads kv head 0, query head 3 reads kv head 1
+    assert oracle.kv_head_of(1, 6, 2) == 0 and oracle.kv_head_of(3, 6, 2) == 1
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_separate(causal):
+    lengths = [5, 1, 17, 9]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    T, H, d = cu[-1], 2, 8
+    q, k, v, do = (_rand((T, H, d), s) for s in (42, 43, 44, 45))
+    O, L = oracle.attn_fwd_varlen(q, k, v, cu, causal, 0.5)
+    dq, dk, dv = oracle.attn_bwd_varlen(q, k, v, do, cu, causal, 0.5)
+    for s in range(len(lengths)):
+        a, e = cu[s], cu[s + 1]
+        Os, Ls = oracle.attn_fwd(q[None, a:e], k[None, a:e], v[None, a:e], causal, 0.5)
+        np.testing.assert_allclose(O[a:e], Os[0], atol=1e-14)
+        np.testing.assert_allclose(L[:, a:e], Ls[0], atol=1e-14)
+        g = oracle.attn_bwd(q[None, a:e], k[None, a:e], v[None, a:e], do[None, a:e], causal, 0.5)
+        for x, y in zip((dq, dk, dv), g):
+            np.testing.assert_allclose(x[a:e], y[0], atol=1e-13)
+
+
+def test_sampled_rows_match_full():
+    q, k, v = _rand((2, 40, 4, 8), 46), _rand((2, 40, 2, 8), 47), _rand((2, 40, 2, 8), 48)
+    rows = synth.sample_rows(0, 40, 4, R=10)
+    O, L = oracle.attn_fwd(q, k, v, True, 0.3)
+    Or, Lr = oracle.attn_fwd_rows(q, k, v, True, 0.3, rows)
+    for h in range(4):
+        np.testing.assert_allclose(Or[:, h], O[:, rows[h], h], atol=1e-14)
+        np.testing.assert_allclose(Lr[:, h], L[:, h, rows[h]], atol=1e-14)
+
+
+def test_merge_partials_reproduces_full():
+    N, d = 29, 8
+    q, k, v = _rand((N, d), 49), _rand((N, d), 50), _rand((N, d), 51)
+    O, L, _ = attention_head(q, k, v, False, 0.4)
+    parts = [(0, 7), (7, 8), (8, 29)]
+    outs, lses = [], []
+    for a, e in parts:
+        o, l, _ = attention_head(q, k[a:e], v[a:e], False, 0.4)
+        outs.append(o)
+        lses.append(l)
+    Om, Lm = oracle.merge_partials(outs, lses)
+    np.testing.assert_allclose(Om, O, atol=1e-12)
+    np.testing.assert_allclose(Lm, L, atol=1e-12)
+
+
+# --- the tiled online-softmax algorithm (C7) --------------------------------
+
+@pytest.mark.parametrize("N,d,bm,bn", [(1, 4, 16, 16), (7, 4, 16, 16), (64, 64, 16, 32), (130, 4, 32, 16),
+                                        (130, 64, 32, 32)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_tiled_equals_untiled(N, d, bm, bn, causal, tau):
+    rng = np.random.default_rng(N * 100 + d)
+    q, k, v = (rng.standard_normal((N, d)) * 3 for _ in range(3))
+    O, L, _ = attention_head(q, k, v, causal, 1 / np.sqrt(d))
+    Ot, Lt = oracle.attn_head_tiled(q, k, v, causal, 1 / np.sqrt(d), bm, bn, tau)
+    np.testing.assert_allclose(Ot, O, atol=1e-12)
+    np.testing.assert_allclose(Lt, L, atol=1e-12)
+
+
+# --- fp8 dequantisation -----------------------------------------------------
+
+def test_dequantize_blockscaled_by_hand():
+    codes = np.zeros((1, 130, 1, 2))
+    codes[0, 0, 0] = [1.0, -2.0]
+    codes[0, 129, 0] = [3.0, 0.5]
+    scales = np.array([[[0.25, 4.0]]])  # block 0 rows 0..127, block 1 rows 128..129
+    x = oracle.dequantize_blockscaled(codes, scales)
+    np.testing.assert_array_equal(x[0, 0, 0], [0.25, -0.5])
+    np.testing.assert_array_equal(x[0, 129, 0], [12.0, 2.0])
+
+
+def test_fp8_synth_roundtrip_error_bounded():
+    """e4m3 has 3 mantissa bits: |x - s*code| <= s * 2**-4 * 2**e for each element."""
+    d = synth.qkv_fp8(0, 1, 256, 2, 2, 64)
+    x = d["q_f32"].astype(np.float64)
+    xh = oracle.dequantize_blockscaled(d["q8"].float(), d["q_scale"])
+    rel = np.abs(x - xh) / np.maximum(np.abs(x), 1e-30)
+    small = np.abs(x) < 2 ** -6 * d["q_scale"].numpy().max()
+    assert np.all(rel[~small] <= 2 ** -4 + 1e-7)
