@@ -1,0 +1,156 @@
+/*
+ * fa_b200 — exact IO-aware scaled dot-product attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation (catalogue record "Dao and colleagues: IO-aware exact
+ * attention with FlashAttention", field summary; topic page "Flash Attention
+ * and Efficient Transformer Mechanisms", opening paragraphs): for every
+ * (sequence b, query head h), with key/value head g = h / (Hq / Hkv),
+ *
+ *     S   = scale * Q[b,:,h,:] K[b,:,g,:]^T      (causal: key j > query i is -inf)
+ *     LSE = logsumexp over keys of S              (natural log, per query row)
+ *     O   = softmax(S) V[b,:,g,:]
+ *
+ * computed tile by tile with an online softmax so the N x N score matrix is
+ * never written to memory; the backward pass recomputes it from Q, K, V and
+ * LSE (the record's summary: recomputation). Nothing is approximated: results
+ * differ from the exact value only by floating-point rounding.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them past the call, and never
+ *    synchronises except in fa_get_status().
+ *  - Layouts are contiguous, row-major:
+ *      padded: Q/O/dO/dQ [B, N, Hq, d], K/V/dK/dV [B, N, Hkv, d]  (BSHD),
+ *              LSE [B, Hq, N] float32;
+ *      packed (varlen): Q/O [T, Hq, d], K/V [T, Hkv, d], LSE [Hq, T];
+ *      sequence s occupies tokens cu_seqlens[s] .. cu_seqlens[s+1]-1.
+ *  - bf16 tensors hold __nv_bfloat16 (IEEE bfloat16); fp8 tensors hold
+ *    __nv_fp8_e4m3 (OCP e4m3, "fn" variant).
+ *  - Data pointers must be 16-byte aligned, LSE 4-byte aligned.
+ *  - Supported head dimensions: d = 64 or 128. Hq must be a multiple of Hkv.
+ *  - Work is launched asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream). Calls are re-entrant; concurrent calls must not
+ *    share output or workspace buffers.
+ *  - Argument errors are reported synchronously, before anything is launched.
+ *    Errors detected on the device (a pipeline wait that gave up) are recorded
+ *    in a per-device status word read by fa_get_status().
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad scale, Hq % Hkv != 0 */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not 64/128, device is not sm_100, size beyond limits */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+  FA_ERR_TIMEOUT = 4,     /* a device-side pipeline wait gave up (see fa_get_status) */
+  FA_ERR_WORKSPACE = 5    /* workspace missing or smaller than fa_bwd_workspace_size() */
+} fa_status_t;
+
+/*
+ * Forward pass, padded batch.
+ *   q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 (in);  o [B,N,Hq,d] bf16 (out);
+ *   lse [B,Hq,N] float32 (out, natural log of the scaled scores' row sums).
+ *   causal: 0 or 1 (query i sees keys 0..i).  scale: > 0 and finite, usually 1/sqrt(d).
+ * B*N == 0 is a no-op returning FA_OK.
+ */
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Forward pass, packed variable-length batch (the varlen API of the
+ * Dao-AILab repository overview).
+ *   q [T,Hq,d], k/v [T,Hkv,d] bf16 (in); o [T,Hq,d] bf16, lse [Hq,T] f32 (out).
+ *   cu_seqlens: DEVICE int32 [nseq+1], non-decreasing, cu_seqlens[0] = 0,
+ *   cu_seqlens[nseq] = total_T. max_seqlen must be >= every sequence length
+ *   (rows beyond it are not computed) and <= 131072.
+ * Each sequence attends only within itself; causal alignment is per sequence.
+ * Output rows of empty sequences are not touched.
+ */
+fa_status_t fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int* cu_seqlens, int nseq, int max_seqlen, int total_T, int Hq, int Hkv, int d,
+                          int causal, float scale, void* stream);
+
+/*
+ * Forward pass with fp8-e4m3 inputs and per-block scales (contribution 3 of
+ * the "FlashAttention-3: Fast and Accurate Attention with Asynchrony and
+ * Low-precision" summary: FP8 GEMMs in the forward pass).
+ *   q8 [B,N,Hq,d], k8/v8 [B,N,Hkv,d] e4m3 codes (in);
+ *   q_scale [B,Hq,ceil(N/128)], k_scale/v_scale [B,Hkv,ceil(N/128)] float32:
+ *   the value of element x of rows 128*i .. 128*i+127 of head h is code * scale[b,h,i].
+ *   o [B,N,Hq,d] bf16, lse [B,Hq,N] float32 (out), as fa_fwd on the dequantised values.
+ *   d must be 128.
+ */
+fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                       const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv,
+                       int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd / fa_bwd_varlen need (fp32 dQ accumulator,
+ * the per-row dot(dO, O) terms and the ordering semaphores). tokens = B*N
+ * (padded) or total_T (varlen); nseq = B or the number of packed sequences.
+ */
+size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
+
+/*
+ * Backward pass, padded batch: gradients of sum(O * dout) with respect to
+ * q, k, v, recomputing the scores from q, k, v and the forward's lse.
+ *   q, k, v, o, dout bf16, lse f32 (in, as produced by fa_fwd);
+ *   dq [B,N,Hq,d], dk/dv [B,N,Hkv,d] bf16 (out; dk/dv summed over the query
+ *   heads of each GQA group).
+ *   workspace: DEVICE buffer of ws_bytes >= fa_bwd_workspace_size(B*N, B, Hq, d),
+ *   16-byte aligned, contents need not be initialised.
+ * The dQ reduction over key blocks is in a fixed order: results are bitwise
+ * reproducible from run to run.
+ */
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq,
+                   int Hkv, int N, int d, int causal, float scale, void* stream);
+
+/* Backward pass, packed variable-length batch; layouts as fa_fwd_varlen. */
+fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                          const int* cu_seqlens, int nseq, int max_seqlen, int total_T, int Hq, int Hkv, int d,
+                          int causal, float scale, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device-side status word
+ * of the current device (FA_OK if no kernel reported an error since the last
+ * call). Returns FA_ERR_CUDA if the synchronisation itself failed.
+ */
+fa_status_t fa_get_status(void* stream);
+
+/* Raw device status word of the last fa_get_status() that found an error
+ * (low byte: status code; bits 8..15: id of the wait that gave up). */
+int fa_last_device_error_word(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* fa_status_string(fa_status_t status);
+
+/*
+ * Upper bound, in nanoseconds, of every device-side pipeline wait of kernels
+ * launched after this call (default 4e9). A wait that runs out records
+ * FA_ERR_TIMEOUT and the kernel exits cleanly instead of hanging.
+ */
+void fa_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Test hook: when set to 1, the next forward launches never load their first
+ * K tile, so the pipeline waits run out and FA_ERR_TIMEOUT is recorded (used
+ * to test the bounded-wait path without faulting the GPU). 0 restores normal
+ * operation.
+ */
+void fa_debug_set_inject(int mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

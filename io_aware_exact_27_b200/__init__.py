@@ -1,0 +1,214 @@
+"""Python binding of libfa_b200 (exact IO-aware attention on B200, sm_100a).
+
+Argument marshalling only: every step of attention runs in the CUDA kernels of
+``libfa_b200.so``; there is no CPU or PyTorch fallback. If the library is
+missing this import fails (build it with ``python -m io_aware_exact_27_b200.build``).
+
+Two layers:
+  * ``fa_fwd``, ``fa_fwd_varlen``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_bwd_varlen``,
+    ``fa_bwd_workspace_size``, ``fa_get_status`` ... — the C entry points of
+    ``include/fa_b200.h`` with the same names and arguments; tensors may be
+    passed as torch CUDA tensors (their data pointers are used) or raw ints.
+    A non-OK status raises ``FAError``.
+  * ``attention_fwd`` / ``attention_fwd_varlen`` / ``attention_bwd`` ... —
+    allocate the outputs with torch on the inputs' device and call the above
+    on the current stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_27_b200.build` "
+                      "(nvcc, sm_100a); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH, mode=ctypes.RTLD_LOCAL)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+_SIGS = {
+    "fa_fwd": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_fwd_varlen": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_fwd_fp8": [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_bwd_varlen": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_get_status": [_P],
+}
+for _name, _args in _SIGS.items():
+    getattr(_lib, _name).argtypes = _args
+    getattr(_lib, _name).restype = _I
+_lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
+_lib.fa_bwd_workspace_size.restype = _Z
+_lib.fa_status_string.argtypes = [_I]
+_lib.fa_status_string.restype = ctypes.c_char_p
+_lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+_lib.fa_set_wait_timeout_ns.restype = None
+_lib.fa_debug_set_inject.argtypes = [_I]
+_lib.fa_debug_set_inject.restype = None
+_lib.fa_last_device_error_word.argtypes = []
+_lib.fa_last_device_error_word.restype = _I
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fa_status_string(status)}")
+
+
+def fa_status_string(status: int) -> str:
+    return _lib.fa_status_string(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != FA_OK:
+        raise FAError(st, where)
+
+
+# ---------------------------------------------------------------- C entry points
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream=None):
+    _check(_lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d, int(causal),
+                       float(scale), _stream(stream)), "fa_fwd")
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total_T, Hq, Hkv, d, causal, scale, stream=None):
+    _check(_lib.fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), nseq, max_seqlen,
+                              total_T, Hq, Hkv, d, int(causal), float(scale), _stream(stream)), "fa_fwd_varlen")
+
+
+def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, N, d, causal, scale, stream=None):
+    _check(_lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _ptr(o),
+                           _ptr(lse), B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)), "fa_fwd_fp8")
+
+
+def fa_bwd_workspace_size(tokens, nseq, Hq, d) -> int:
+    return int(_lib.fa_bwd_workspace_size(tokens, nseq, Hq, d))
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N, d, causal, scale, stream=None):
+    _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                       _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)),
+           "fa_bwd")
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total_T,
+                  Hq, Hkv, d, causal, scale, stream=None):
+    _check(_lib.fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                              _ptr(dv), _ptr(workspace), ws_bytes, _ptr(cu_seqlens), nseq, max_seqlen, total_T, Hq,
+                              Hkv, d, int(causal), float(scale), _stream(stream)), "fa_bwd_varlen")
+
+
+def fa_get_status(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status code."""
+    return int(_lib.fa_get_status(_stream(stream)))
+
+
+def fa_last_device_error_word() -> int:
+    return int(_lib.fa_last_device_error_word())
+
+
+def fa_set_wait_timeout_ns(ns: int):
+    _lib.fa_set_wait_timeout_ns(int(ns))
+
+
+def fa_debug_set_inject(mode: int):
+    _lib.fa_debug_set_inject(int(mode))
+
+
+# ---------------------------------------------------------------- torch conveniences
+
+def _default_scale(d, scale):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def attention_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 CUDA tensors -> (o [B,N,Hq,d] bf16, lse [B,Hq,N] f32)."""
+    import torch
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, _default_scale(d, scale), stream)
+    return o, lse
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, scale=None, out=None, lse=None,
+                         stream=None):
+    """q [T,Hq,d], k/v [T,Hkv,d] bf16, cu_seqlens int32 [nseq+1] (CUDA) -> (o [T,Hq,d], lse [Hq,T])."""
+    import torch
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, cu_seqlens.numel() - 1, max_seqlen, T, Hq, Hkv, d, causal,
+                  _default_scale(d, scale), stream)
+    return o, lse
+
+
+def attention_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None, stream=None):
+    """e4m3 q8 [B,N,Hq,d], k8/v8 [B,N,Hkv,d] + f32 block scales -> (o bf16, lse f32)."""
+    import torch
+    B, N, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, N, d, causal, _default_scale(d, scale),
+               stream)
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(o * dout); inputs as attention_fwd produced them."""
+    import torch
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B * N, B, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), B, Hq, Hkv, N, d, causal,
+           _default_scale(d, scale), stream)
+    return dq, dk, dv
+
+
+def attention_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, causal=False, scale=None, workspace=None,
+                         stream=None):
+    import torch
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(T, nseq, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), cu_seqlens, nseq, max_seqlen, T,
+                  Hq, Hkv, d, causal, _default_scale(d, scale), stream)
+    return dq, dk, dv

@@ -1,0 +1,249 @@
+// C-ABI of the attention library: argument validation, TMA tensor-map
+// encoding, launch configuration and the device status word. The kernels
+// live in the fa_*_kernel.cuh headers included below (one translation unit).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa_b200.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+__device__ int g_status_word;  // first device-side error since the last fa_get_status()
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::atomic<uint64_t> g_timeout_ns{4000000000ull};
+std::atomic<int> g_inject{0};
+std::atomic<int> g_last_word{0};
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int cc = 0;
+  int* status = nullptr;     // device address of g_status_word
+  bool fwd_attr[2] = {false, false};
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// Per-device facts, looked up once per device with that device current.
+fa_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return FA_ERR_CUDA;
+    s.cc = major * 10 + minor;
+    s.sms = sms;
+    s.status = static_cast<int*>(p);
+    s.ready = true;
+  }
+  if (s.cc != 100) return FA_ERR_UNSUPPORTED;
+  *out = &s;
+  return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// [tokens, heads, d] tensor with 128-row x 64-element (128-byte) boxes, 128B swizzle.
+fa_status_t encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int tokens,
+                        int heads, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const int box_inner = 128 / elem_bytes;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes,
+                           static_cast<cuuint64_t>(heads) * d * elem_bytes};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, 128};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int Hq,
+                         int Hkv, int d, float scale) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+template <int D>
+fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, fa::FwdArgs a, int tokens,
+                       long long units_bound, cudaStream_t stream) {
+  constexpr int STAGES = 4;
+  using Smem = fa::FwdSmem<D, STAGES>;
+  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES>;
+  const int smem = static_cast<int>(sizeof(Smem)) + 1024;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    bool& done = ds->fwd_attr[D == 128 ? 1 : 0];
+    if (!done) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return FA_ERR_CUDA;
+      done = true;
+    }
+  }
+  CUtensorMap tq, tk, tv;
+  fa_status_t st;
+  if ((st = encode_rows(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hq, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  a.timeout_ns = g_timeout_ns.load();
+  a.inject = g_inject.load();
+  a.status = ds->status;
+  const int grid = static_cast<int>(units_bound < ds->sms ? units_bound : ds->sms);
+  if (grid <= 0) return FA_OK;
+  kern<<<grid, fa::kThreadsFwd, smem, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int nseq,
+                         int N, int total_T, int Hq, int Hkv, int d, int causal, float scale, void* stream) {
+  fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
+  if (st != FA_OK) return st;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  fa::FwdArgs a{};
+  a.o = o;
+  a.lse = lse;
+  a.cu_seqlens = cu;
+  a.nseq = nseq;
+  a.N = N;
+  a.total_T = total_T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const long long nlev = (N + 255) / 256;
+  long long bound;
+  if (cu == nullptr) {
+    a.lse_head_stride = N;
+    bound = static_cast<long long>(nseq) * Hq * nlev;
+    a.num_units = static_cast<int>(bound);
+  } else {
+    a.lse_head_stride = total_T;
+    const long long by_len = static_cast<long long>(nseq) * nlev;
+    const long long by_tok = (static_cast<long long>(total_T) + 255) / 256 + nseq;
+    bound = static_cast<long long>(Hq) * (by_len < by_tok ? by_len : by_tok);
+    a.num_units = static_cast<int>(bound);  // recomputed exactly on the device
+  }
+  if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_fwd<128>(ds, q, k, v, a, total_T, bound, s)
+                  : launch_fwd<64>(ds, q, k, v, a, total_T, bound, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                   int d, int causal, float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  return fwd_dispatch(q, k, v, o, lse, nullptr, B, N, B * N, Hq, Hkv, d, causal, scale, stream);
+}
+
+fa_status_t fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                          int nseq, int max_seqlen, int total_T, int Hq, int Hkv, int d, int causal, float scale,
+                          void* stream) {
+  if (nseq < 0 || total_T < 0 || max_seqlen < 0 || cu_seqlens == nullptr || !aligned(cu_seqlens, 4))
+    return FA_ERR_INVALID_ARG;
+  if (nseq == 0 || total_T == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > 131072) return FA_ERR_UNSUPPORTED;
+  return fwd_dispatch(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total_T, Hq, Hkv, d, causal, scale, stream);
+}
+
+fa_status_t fa_fwd_fp8(const void*, const void*, const void*, const float*, const float*, const float*, void*,
+                       float*, int, int, int, int, int, int, float, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
+  if (tokens <= 0 || Hq <= 0 || d <= 0 || nseq < 0) return 0;
+  const size_t dq_acc = static_cast<size_t>(tokens) * Hq * d * sizeof(float);
+  const size_t dterm = static_cast<size_t>(tokens) * Hq * sizeof(float);
+  const size_t sems = (static_cast<size_t>(tokens) / 128 + static_cast<size_t>(nseq) + 1) * Hq * sizeof(int);
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  return up(dq_acc) + up(dterm) + up(sems);
+}
+
+fa_status_t fa_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
+                   void*, void*, size_t, int, int, int, int, int, int, float, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+fa_status_t fa_bwd_varlen(const void*, const void*, const void*, const void*, const float*, const void*, void*,
+                          void*, void*, void*, size_t, const int*, int, int, int, int, int, int, int, float, void*) {
+  return FA_ERR_UNSUPPORTED;
+}
+
+fa_status_t fa_get_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_status_word, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (w == 0) return FA_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  g_last_word.store(w);
+  return static_cast<fa_status_t>(w & 0xff);
+}
+
+int fa_last_device_error_word(void) { return g_last_word.load(); }
+
+const char* fa_status_string(fa_status_t s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
+
+void fa_debug_set_inject(int mode) { g_inject.store(mode); }
+
+}  // extern "C"

@@ -1,0 +1,409 @@
+// Forward pass of exact attention on sm_100a (bf16 in, fp32 accumulation).
+//
+// What it computes: O = softmax(scale * Q K^T + mask) V and the per-row
+// natural-log LSE, tile by tile, the score matrix living only in tensor
+// memory (catalogue record "Dao and colleagues: IO-aware exact attention with
+// FlashAttention", summary: exact attention without materialising the full
+// attention matrix; Dao-AILab repository overview: online softmax with
+// rescaling, tiled attention, persistent tile schedulers).
+//
+// Design (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax of query tile 0 (thread = row = TMEM lane)
+//   warps 4-7  softmax of query tile 1
+//   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a ring
+//   warp  9    tcgen05 issuer (one thread) and TMEM owner
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+// P (bf16) is written over the first 64 columns of its S tile and fed to the
+// PV MMA straight from TMEM. The two query tiles ping-pong: while one tile's
+// softmax runs, the tensor core works on the other tile's GEMMs.
+#pragma once
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;      // query rows per tile
+constexpr int kBN = 128;      // keys per block
+constexpr int kThreadsFwd = 320;
+constexpr float kTau = 8.0f;  // lazy-rescale threshold, base-2 exponent units
+
+struct FwdArgs {
+  void* o;
+  float* lse;
+  const int* cu_seqlens;
+  int nseq;        // padded: B
+  int N;           // padded: N; varlen: max_seqlen
+  int total_T;     // tokens in the packed token dimension
+  int Hq, Hkv;
+  int causal;
+  float scale;     // softmax scale
+  float scale_log2;  // scale * log2(e)
+  int lse_head_stride;  // padded: N; varlen: total_T
+  int num_units;   // padded: exact; varlen: upper bound
+  uint64_t timeout_ns;
+  int* status;
+  int inject;      // test hook: 1 = the producer never loads the first K tile
+};
+
+template <int D, int STAGES>
+struct FwdSmem {
+  static constexpr int kTileBytes = kBM * D * 2;  // one 128 x D bf16 tile
+  alignas(1024) uint8_t q[2][kTileBytes];
+  alignas(1024) uint8_t kv[STAGES][kTileBytes];
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[STAGES], kv_empty[STAGES];
+  uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int level_count[512];
+};
+
+// Loads one 128 x D bf16 tile as D/64 boxes of 128 rows x 128 bytes (SW128).
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m, uint32_t bar, int head, int row0) {
+#pragma unroll
+  for (int b = 0; b < D / 64; ++b) tma_load_3d(dst + b * 16384, m, bar, b * 64, head, row0);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_f16_ss(s_tmem, smem_desc(q_smem + off, 16, 1024, kSwizzle128B),
+               smem_desc(k_smem + off, 16, 1024, kSwizzle128B), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    // V tile is [keys, D] (D contiguous): MN-major B operand; LBO = next 64
+    // columns of D (next TMA box), SBO = next 8 keys.
+    mma_f16_ts(o_tmem, p_tmem + kk * 8, smem_desc(v_smem + kk * 2048, 16384, 1024, kSwizzle128B), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
+  const int nb = (u.n + kBN - 1) / kBN;
+  return causal ? min(nb, 2 * u.qb2 + 2) : nb;
+}
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreadsFwd, 1)
+    fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
+  using Smem = FwdSmem<D, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // ---- set-up: barriers, TMEM, varlen level table
+  if (tid == 0) {
+    mbar_init(smem_u32(&sm.q_full), 1);
+    mbar_init(smem_u32(&sm.q_empty), 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&sm.kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.s_full[i]), 1);
+      mbar_init(smem_u32(&sm.p_full[i]), 128);
+      mbar_init(smem_u32(&sm.o_final[i]), 1);
+      mbar_init(smem_u32(&sm.o_free[i]), 128);
+    }
+    mbar_init(smem_u32(&sm.drain), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  const int nlevels = (args.N + 255) / 256;
+  const bool varlen = args.cu_seqlens != nullptr;
+  if (varlen) {
+    for (int L = tid; L < nlevels; L += kThreadsFwd) sm.level_count[L] = 0;
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  __syncthreads();
+  int num_units = args.num_units;
+  if (varlen) {
+    for (int s = tid; s < args.nseq; s += kThreadsFwd) {
+      const int n = __ldg(args.cu_seqlens + s + 1) - __ldg(args.cu_seqlens + s);
+      const int nl = min((n + 255) >> 8, nlevels);
+      for (int L = 0; L < nl; ++L) atomicAdd(&sm.level_count[L], 1);
+    }
+    __syncthreads();
+    int tot = 0;
+    for (int L = 0; L < nlevels; ++L) tot += sm.level_count[L];
+    num_units = tot * args.Hq;
+  }
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, args.causal, nlevels, sm.level_count};
+  const volatile int* abort = &sm.abort;
+  const int group = args.Hq / args.Hkv;
+  uint32_t prod_issued = 0;  // K/V loads issued by the producer thread
+  uint32_t q_issued = 0;     // Q loads issued by the producer thread
+
+  if (warp == 8) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      uint32_t kv_prod = 0, it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+        const Unit un = decode_unit(sched, u);
+        const int nblk = num_kv_blocks(un, args.causal);
+        const int hkv = un.h / group;
+        if (!mbar_wait(smem_u32(&sm.q_empty), (it & 1) ^ 1, abort, args.timeout_ns)) {
+          report_error(args.status, kStatusTimeout, 1);
+          ok = false;
+          break;
+        }
+        const uint32_t qbar = smem_u32(&sm.q_full);
+        mbar_expect_tx(qbar, 2 * Smem::kTileBytes);
+        const int row0 = un.tok0 + un.qb2 * 2 * kBM;
+        load_tile<D>(smem_u32(sm.q[0]), &tm_q, qbar, un.h, row0);
+        load_tile<D>(smem_u32(sm.q[1]), &tm_q, qbar, un.h, row0 + kBM);
+        q_issued = it + 1;
+        for (int j = 0; j < nblk && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = kv_prod % STAGES;
+            if (!mbar_wait(smem_u32(&sm.kv_empty[slot]), ((kv_prod / STAGES) & 1) ^ 1, abort, args.timeout_ns)) {
+              report_error(args.status, kStatusTimeout, 2);
+              ok = false;
+              break;
+            }
+            if (args.inject == 1 && it == 0 && j == 0 && kv == 0) {
+              // test hook: the first K tile of the unit is never loaded
+            } else {
+              const uint32_t bar = smem_u32(&sm.kv_full[slot]);
+              mbar_expect_tx(bar, Smem::kTileBytes);
+              load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
+            }
+            ++kv_prod;
+          }
+        }
+      }
+      if (!ok) sm.abort = 1;
+      prod_issued = kv_prod;
+    }
+  } else if (warp == 9) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      uint32_t kv_cons = 0, it = 0, pc0 = 0, pc1 = 0;
+      bool ok = true;
+      const uint32_t S0 = tmem + 0, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 384;
+      auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        if (!mbar_wait(smem_u32(bar), parity, abort, args.timeout_ns)) {
+          report_error(args.status, kStatusTimeout, site);
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+        const Unit un = decode_unit(sched, u);
+        const int nblk = num_kv_blocks(un, args.causal);
+        if (!(ok = wait(&sm.q_full, it & 1, 10))) break;
+        const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
+        uint32_t slotK = kv_cons % STAGES;
+        if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 11))) break;
+        ++kv_cons;
+        issue_qk<D>(S0, q0, smem_u32(sm.kv[slotK]));
+        tc_commit(smem_u32(&sm.s_full[0]));
+        issue_qk<D>(S1, q1, smem_u32(sm.kv[slotK]));
+        tc_commit(smem_u32(&sm.s_full[1]));
+        tc_commit(smem_u32(&sm.kv_empty[slotK]));
+        if (nblk == 1) tc_commit(smem_u32(&sm.q_empty));
+        for (int j = 0; j < nblk; ++j) {
+          const bool has_next = j + 1 < nblk;
+          const uint32_t slotV = kv_cons % STAGES;
+          if (!(ok = wait(&sm.kv_full[slotV], (kv_cons / STAGES) & 1, 12))) break;
+          ++kv_cons;
+          if (has_next) {
+            slotK = kv_cons % STAGES;
+            if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 13))) break;
+            ++kv_cons;
+          }
+          const uint32_t vaddr = smem_u32(sm.kv[slotV]);
+          // ---- tile 0
+          if (!(ok = wait(&sm.p_full[0], pc0 & 1, 14))) break;
+          ++pc0;
+          if (j == 0 && !(ok = wait(&sm.o_free[0], (it & 1) ^ 1, 15))) break;
+          issue_pv<D>(O0, S0, vaddr, j > 0);
+          if (has_next) {
+            issue_qk<D>(S0, q0, smem_u32(sm.kv[slotK]));
+            tc_commit(smem_u32(&sm.s_full[0]));
+          } else {
+            tc_commit(smem_u32(&sm.o_final[0]));
+          }
+          // ---- tile 1
+          if (!(ok = wait(&sm.p_full[1], pc1 & 1, 16))) break;
+          ++pc1;
+          if (j == 0 && !(ok = wait(&sm.o_free[1], (it & 1) ^ 1, 17))) break;
+          issue_pv<D>(O1, S1, vaddr, j > 0);
+          tc_commit(smem_u32(&sm.kv_empty[slotV]));
+          if (has_next) {
+            issue_qk<D>(S1, q1, smem_u32(sm.kv[slotK]));
+            tc_commit(smem_u32(&sm.s_full[1]));
+            tc_commit(smem_u32(&sm.kv_empty[slotK]));
+            if (j + 2 == nblk) tc_commit(smem_u32(&sm.q_empty));
+          } else {
+            tc_commit(smem_u32(&sm.o_final[1]));
+          }
+        }
+      }
+      if (!ok) sm.abort = 1;
+      // every MMA issued so far must finish before TMEM is released
+      tc_commit(smem_u32(&sm.drain));
+      mbar_wait(smem_u32(&sm.drain), 0, nullptr, args.timeout_ns);
+    }
+  } else {
+    // ======================= softmax warpgroups =======================
+    const int tile = warp >> 2;               // 0 or 1
+    const int quad = warp & 3;                // TMEM lane quadrant
+    const int r_in_tile = quad * 32 + lane;   // TMEM lane = row within the tile
+    const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t S = tmem + tile * 128 + lane_bits;
+    const uint32_t O = tmem + 256 + tile * 128 + lane_bits;
+    const float cl = args.scale_log2;
+    uint32_t sc = 0, it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+      const Unit un = decode_unit(sched, u);
+      const int nblk = num_kv_blocks(un, args.causal);
+      const int row = un.qb2 * 2 * kBM + tile * kBM + r_in_tile;  // row within the sequence
+      const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;  // last visible key
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nblk; ++j) {
+        // every lane waits; the outcome is made warp-uniform so that the
+        // warp-collective tcgen05 loads below run converged
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[tile]), sc & 1, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 20 + tile);
+          break;
+        }
+        ++sc;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(S + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(S + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(S + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        float* s = reinterpret_cast<float*>(sr);
+        const int kv0 = j * kBN;
+        if (kv0 + kBN - 1 > limit) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (kv0 + c > limit) s[c] = -INFINITY;
+        }
+        float mt = s[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+        const bool need = (mt - m) * cl > kTau;
+        const float m_new = need ? mt : m;
+        const float alpha = need ? ex2_approx((m - m_new) * cl) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O rows whose maximum moved are rescaled in TMEM; the PV MMA of
+          // the previous block has completed (it precedes this S in issue
+          // order), so O is quiescent here.
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t orr[32];
+            tmem_ld32(O + c, orr);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) orr[t] = __float_as_uint(__uint_as_float(orr[t]) * alpha);
+            tmem_st32(O + c, orr);
+          }
+        }
+        const float mc = m_new * cl;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float p0 = ex2_approx(fmaf(s[c4 * 32 + 2 * t], cl, -mc));
+            const float p1 = ex2_approx(fmaf(s[c4 * 32 + 2 * t + 1], cl, -mc));
+            lsum += p0 + p1;
+            pk[t] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(S + c4 * 16, pk);
+        }
+        l = l * alpha + lsum;
+        m = m_new;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.p_full[tile]));
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, LSE
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[tile]), it & 1, abort, args.timeout_ns));
+      if (!ok) {
+        if (lane == 0) report_error(args.status, kStatusTimeout, 22 + tile);
+        break;
+      }
+      tc_fence_after();
+      const bool valid = row < un.n;
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
+                            (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t orr[32];
+        tmem_ld32(O + c, orr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          pk[t] = pack_bf16x2(__uint_as_float(orr[2 * t]) * inv_l, __uint_as_float(orr[2 * t + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.o_free[tile]));
+      if (valid) {
+        const size_t li = varlen ? (static_cast<size_t>(un.h) * args.lse_head_stride + un.tok0 + row)
+                                 : (static_cast<size_t>(un.seq * args.Hq + un.h) * args.lse_head_stride + row);
+        args.lse[li] = m * args.scale + logf(l);
+      }
+    }
+    if (!ok) sm.abort = 1;
+  }
+
+  // ---- teardown: every role is out of its loop; release TMEM
+  tc_fence_before();
+  __syncthreads();
+  if (sm.abort && warp == 8 && lane == 0) {
+    // after an abort, let the K/V loads already issued land before the CTA
+    // exits (the newest load of each ring slot is the one still in flight)
+    for (uint32_t i = (prod_issued > STAGES ? prod_issued - STAGES : 0); i < prod_issued; ++i) {
+      if (args.inject == 1 && i == 0) continue;  // never issued
+      mbar_wait(smem_u32(&sm.kv_full[i % STAGES]), (i / STAGES) & 1, nullptr, args.timeout_ns);
+    }
+    if (q_issued > 0) mbar_wait(smem_u32(&sm.q_full), (q_issued - 1) & 1, nullptr, args.timeout_ns);
+  }
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa
