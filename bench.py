@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention hot path on B200 (attention TFLOP/s).
+
+One step = the whole hot path over one batch of synthetic input: the causal
+bf16 forward pass (O, LSE) and, when the library provides it, the backward
+pass (dQ, dK, dV) on the workload B=4, Hq=Hkv=16, N=2048, d=128 (Q, K, V, dO
+i.i.d. N(0,1) rounded to bf16, seed 0). Flops: forward 4*B*Hq*N^2*d halved for
+causal, backward 2.5x the forward (five GEMMs instead of two).
+
+Prints ONE JSON line (rank 0). `--impl reference` times the fp64 CPU oracle
+instead, on a bounded sample of the same workload. Multi-GPU (torchrun):
+every rank runs its own independent batch (weak scaling, no data-path
+collective); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = {"workload": "bf16 causal attention fwd+bwd, B=4 Hq=Hkv=16 N=2048 d=128",
+            "B": 4, "Hq": 16, "Hkv": 16, "N": 2048, "d": 128, "causal": True}
+METRIC = "attention TFLOP/s (bf16/fp8, causal, N=2K–16K) and % of B200 tensor peak"
+UNIT = "TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def fwd_flops(B, Hq, N, d, causal):
+    return 4.0 * B * Hq * N * N * d / (2.0 if causal else 1.0)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-bwd", action="store_true", help="time the forward pass only")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {"bf16_tflops": j["bf16_tflops"], "bf16_tflops_sustained": j["bf16_tflops_sustained"],
+                "hbm_gbs": j["hbm_gbs"], "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    csrc = os.path.join(ROOT, "io_aware_exact_27_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    when the kernel sources changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    e = j.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        mhz.sort()
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------- reference arm (CPU oracle)
+
+def oracle_sample(budget_s, with_bwd):
+    """Times the fp64 oracle on whole (batch, head) problems of the workload
+    until `budget_s` is spent; returns (TFLOP/s, heads done, seconds, cores)."""
+    import numpy as np
+    import oracle
+    import synth
+    w = WORKLOAD
+    q, k, v, do = synth.qkv_bf16(0, w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], with_dout=True)
+    scale = 1.0 / math.sqrt(w["d"])
+    per_head = fwd_flops(1, 1, w["N"], w["d"], True) * (3.5 if with_bwd else 1.0)
+    done, t0 = 0, time.perf_counter()
+    total = w["B"] * w["Hq"]
+    while done < total:
+        b, h = divmod(done, w["Hq"])
+        g = oracle.kv_head_of(h, w["Hq"], w["Hkv"])
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        slk = (slice(b, b + 1), slice(None), slice(g, g + 1))
+        oracle.attn_fwd(q[sl], k[slk], v[slk], True, scale)
+        if with_bwd:
+            oracle.attn_bwd(q[sl], k[slk], v[slk], do[sl], True, scale)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    cores = os.cpu_count()
+    return per_head * done / el / 1e12, done, el, cores
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    with_bwd = not args.no_bwd
+    # each step: a bounded sample sized so the whole run ends within minutes
+    per_step_budget = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, heads, el, cores = oracle_sample(per_step_budget, with_bwd)
+        if i >= args.warmup:
+            vals.append((tf, heads, el))
+    tf = sum(v[0] for v in vals) / len(vals)
+    ms = sum(v[2] for v in vals) / len(vals) * 1e3
+    heads = vals[-1][1]
+    total = WORKLOAD["B"] * WORKLOAD["Hq"]
+    sample = f"{heads} of {total} (batch, head) problems per step, fp64 numpy, {'fwd+bwd' if with_bwd else 'fwd'}"
+    line = {"metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": dict(WORKLOAD, parallelism=f"replicas{args.gpus}", l2="n/a (CPU)"),
+            "cpu_baseline": {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    import synth
+
+    w = WORKLOAD
+    B, Hq, Hkv, N, d, causal = w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], w["causal"]
+    scale = 1.0 / math.sqrt(d)
+    with_bwd = not args.no_bwd
+    if with_bwd:
+        try:
+            probe_ws = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+            fa.fa_bwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, probe_ws, B, Hq, Hkv, N, d, 1, scale)
+        except fa.FAError as e:
+            if e.status == fa.FA_ERR_UNSUPPORTED:
+                with_bwd = False  # backward not in this build of the library
+    q_h, k_h, v_h, do_h = synth.qkv_bf16(rank, B, N, Hq, Hkv, d, with_dout=True)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def step():
+        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+        if with_bwd:
+            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale, sptr)
+
+    launches_per_step = 1 + (3 if with_bwd else 0)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+
+    # timed region: K steps, L2 flushed before each (outside the step's events)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            a, mid, b = ev[i]
+            a.record(stream)
+            fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+            mid.record(stream)
+            if with_bwd:
+                fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale, sptr)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    st = fa.fa_get_status(sptr)
+    if st != fa.FA_OK:
+        raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
+    step_ms = [a.elapsed_time(b) for a, _, b in ev]
+    fwd_ms = [a.elapsed_time(m) for a, m, _ in ev]
+    bwd_ms = [m.elapsed_time(b) for _, m, b in ev]
+    tot_ms = sum(step_ms)
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms_per_step = tot_ms / args.steps
+    f_fwd = fwd_flops(B, Hq, N, d, causal)
+    f_step = f_fwd * (3.5 if with_bwd else 1.0)
+    value = f_step * world * args.steps / (tot_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (largest share of the step)
+    pk = peaks()
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    bwd_avg = sum(bwd_ms) / len(bwd_ms) if with_bwd else 0.0
+    if with_bwd and bwd_avg > fwd_avg:
+        dom, dom_flops, dom_ms = "fa_bwd", 2.5 * f_fwd, bwd_avg
+    else:
+        dom, dom_flops, dom_ms = "fa_fwd_sm100_kernel", f_fwd, fwd_avg
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for(dom),
+                "peak_source": f"{pk['source']} bf16 burst (cuBLAS)",
+                "fwd_ms": fwd_avg, "bwd_ms": bwd_avg if with_bwd else None}
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in (pin if with_bwd else pin[:3]))
+        d2h = sum(t.numel() * t.element_size() for t in (outs_h if with_bwd else outs_h[:2]))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            q.copy_(pin[0], non_blocking=True)
+            k.copy_(pin[1], non_blocking=True)
+            v.copy_(pin[2], non_blocking=True)
+            if with_bwd:
+                do.copy_(pin[3], non_blocking=True)
+            step()
+            outs_h[0].copy_(o, non_blocking=True)
+            outs_h[1].copy_(lse, non_blocking=True)
+            if with_bwd:
+                outs_h[2].copy_(dq, non_blocking=True)
+                outs_h[3].copy_(dk, non_blocking=True)
+                outs_h[4].copy_(dv, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": f_step * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, heads, el, cores = oracle_sample(args.cpu_budget_s, with_bwd)
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{heads} of {B * Hq} (batch, head) problems of the workload, fp64 numpy, "
+                         f"{'fwd+bwd' if with_bwd else 'fwd'}, {el:.1f} s"}
+
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = dict(WORKLOAD)
+    cfg["workload"] = WORKLOAD["workload"] if with_bwd else WORKLOAD["workload"].replace("fwd+bwd", "fwd")
+    cfg.update({"parallelism": f"dp{world}" if world > 1 else "single", "l2": "flushed before every step",
+                "global_batch": B * world})
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps if with_bwd else args.steps,
+            "pct_of_peak": value / world / pk["bf16_tflops"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
