@@ -47,7 +47,15 @@ def parse():
     ap.add_argument("--no-bwd", action="store_true", help="time the forward pass only")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
-    return ap.parse_args()
+    ap.add_argument("--shape", default=None,
+                    help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
+    args = ap.parse_args()
+    if args.shape:
+        B, Hq, Hkv, N, d, c = (int(x) for x in args.shape.split(","))
+        WORKLOAD.update({"B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": bool(c),
+                         "workload": f"bf16 {'causal' if c else 'non-causal'} attention fwd+bwd, "
+                                     f"B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}"})
+    return args
 
 
 def peaks():
@@ -148,7 +156,7 @@ def oracle_sample(budget_s, with_bwd):
     w = WORKLOAD
     q, k, v, do = synth.qkv_bf16(0, w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], with_dout=True)
     scale = 1.0 / math.sqrt(w["d"])
-    per_head = fwd_flops(1, 1, w["N"], w["d"], True) * (3.5 if with_bwd else 1.0)
+    per_head = fwd_flops(1, 1, w["N"], w["d"], w["causal"]) * (3.5 if with_bwd else 1.0)
     done, t0 = 0, time.perf_counter()
     total = w["B"] * w["Hq"]
     while done < total:
@@ -156,9 +164,9 @@ def oracle_sample(budget_s, with_bwd):
         g = oracle.kv_head_of(h, w["Hq"], w["Hkv"])
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
         slk = (slice(b, b + 1), slice(None), slice(g, g + 1))
-        oracle.attn_fwd(q[sl], k[slk], v[slk], True, scale)
+        oracle.attn_fwd(q[sl], k[slk], v[slk], w["causal"], scale)
         if with_bwd:
-            oracle.attn_bwd(q[sl], k[slk], v[slk], do[sl], True, scale)
+            oracle.attn_bwd(q[sl], k[slk], v[slk], do[sl], w["causal"], scale)
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -235,9 +243,9 @@ def run_ours(args):
     sptr = stream.cuda_stream
 
     def step():
-        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
         if with_bwd:
-            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale, sptr)
+            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, int(causal), scale, sptr)
 
     launches_per_step = 1 + (3 if with_bwd else 0)
     for _ in range(args.warmup):
@@ -257,10 +265,10 @@ def run_ours(args):
             flush.zero_()
             a, mid, b = ev[i]
             a.record(stream)
-            fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+            fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
             mid.record(stream)
             if with_bwd:
-                fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale, sptr)
+                fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, int(causal), scale, sptr)
             b.record(stream)
         torch.cuda.synchronize(dev)
     if pg:

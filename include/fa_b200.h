@@ -93,9 +93,10 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
                        int N, int d, int causal, float scale, void* stream);
 
 /*
- * Bytes of device workspace fa_bwd / fa_bwd_varlen need (fp32 dQ accumulator,
- * the per-row dot(dO, O) terms and the ordering semaphores). tokens = B*N
- * (padded) or total_T (varlen); nseq = B or the number of packed sequences.
+ * Bytes of device workspace fa_bwd / fa_bwd_varlen need: two fp32 vectors per
+ * (query head, token), the row's LSE in base 2 and D = dot(dO, O), with 128
+ * padding rows per head. tokens = B*N (padded) or total_T (varlen); nseq and
+ * d do not change the size (kept for a stable signature). 0 for empty inputs.
  */
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
 
@@ -106,9 +107,11 @@ size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
  *   dq [B,N,Hq,d], dk/dv [B,N,Hkv,d] bf16 (out; dk/dv summed over the query
  *   heads of each GQA group).
  *   workspace: DEVICE buffer of ws_bytes >= fa_bwd_workspace_size(B*N, B, Hq, d),
- *   16-byte aligned, contents need not be initialised.
- * The dQ reduction over key blocks is in a fixed order: results are bitwise
- * reproducible from run to run.
+ *   256-byte aligned, contents need not be initialised (FA_ERR_WORKSPACE
+ *   otherwise).
+ * No atomics: every gradient element is produced by one CTA in a fixed
+ * order, so results are bitwise reproducible from run to run. Three kernels
+ * run on `stream`: the D/LSE preparation, dK/dV, and dQ.
  */
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq,
@@ -148,6 +151,16 @@ void fa_set_wait_timeout_ns(uint64_t ns);
  * operation.
  */
 void fa_debug_set_inject(int mode);
+
+/*
+ * Tuning knob of the bf16 forward kernels: of every 8 pairs of score
+ * elements, how many take their exponential on the FMA pipe (a cubic
+ * polynomial after exact range reduction, relative error < 1e-4) instead of
+ * the MUFU unit, which otherwise limits the softmax. Accepted: 0, 2, 3
+ * (default 2); other values return FA_ERR_UNSUPPORTED. Blocks that contain
+ * masked keys always use MUFU. Affects launches made after the call.
+ */
+fa_status_t fa_set_exp_emulation(int pairs_of_8);
 
 #ifdef __cplusplus
 }

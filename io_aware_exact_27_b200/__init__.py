@@ -2,7 +2,7 @@
 
 Argument marshalling only: every step of attention runs in the CUDA kernels of
 ``libfa_b200.so``; there is no CPU or PyTorch fallback. If the library is
-missing this import fails (build it with ``python -m io_aware_exact_27_b200.build``).
+missing this import fails (build it with ``python io_aware_exact_27_b200/build.py``).
 
 Two layers:
   * ``fa_fwd``, ``fa_fwd_varlen``, ``fa_fwd_fp8``, ``fa_bwd``, ``fa_bwd_varlen``,
@@ -25,7 +25,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_27_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python io_aware_exact_27_b200/build.py` "
                       "(nvcc, sm_100a); there is no fallback implementation")
 
 _lib = ctypes.CDLL(LIB_PATH, mode=ctypes.RTLD_LOCAL)
@@ -42,6 +42,7 @@ _SIGS = {
     "fa_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_varlen": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_get_status": [_P],
+    "fa_set_exp_emulation": [_I],
 }
 for _name, _args in _SIGS.items():
     getattr(_lib, _name).argtypes = _args
@@ -137,6 +138,10 @@ def fa_last_device_error_word() -> int:
 
 def fa_set_wait_timeout_ns(ns: int):
     _lib.fa_set_wait_timeout_ns(int(ns))
+
+
+def fa_set_exp_emulation(pairs_of_8: int):
+    _check(_lib.fa_set_exp_emulation(int(pairs_of_8)), "fa_set_exp_emulation")
 
 
 def fa_debug_set_inject(mode: int):

@@ -10,7 +10,7 @@
 #include <mutex>
 
 #include "../../include/fa_b200.h"
-#include "fa_fwd_kernel.cuh"
+#include "fa_bwd_kernel.cuh"
 
 namespace {
 
@@ -22,6 +22,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 std::atomic<int> g_inject{0};
+std::atomic<int> g_exp_emu{2};  // pairs of every 8 whose exp2 runs on the FMA pipe
 std::atomic<int> g_last_word{0};
 
 constexpr int kMaxDevices = 64;
@@ -31,7 +32,8 @@ struct DeviceState {
   int sms = 0;
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
-  bool fwd_attr[2] = {false, false};
+  bool fwd_attr[2][5] = {};
+  bool bwd_attr[2] = {false, false};
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -103,16 +105,16 @@ fa_status_t check_common(const void* q, const void* k, const void* v, const void
   return FA_OK;
 }
 
-template <int D>
+template <int D, int EMU>
 fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, fa::FwdArgs a, int tokens,
                        long long units_bound, cudaStream_t stream) {
   constexpr int STAGES = 4;
   using Smem = fa::FwdSmem<D, STAGES>;
-  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES>;
+  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU>;
   const int smem = static_cast<int>(sizeof(Smem)) + 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->fwd_attr[D == 128 ? 1 : 0];
+    bool& done = ds->fwd_attr[D == 128 ? 1 : 0][EMU];
     if (!done) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -167,8 +169,117 @@ fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, f
   }
   if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_fwd<128>(ds, q, k, v, a, total_T, bound, s)
-                  : launch_fwd<64>(ds, q, k, v, a, total_T, bound, s);
+  switch ((d == 128 ? 10 : 0) + g_exp_emu.load()) {
+    case 0: return launch_fwd<64, 0>(ds, q, k, v, a, total_T, bound, s);
+    case 2: return launch_fwd<64, 2>(ds, q, k, v, a, total_T, bound, s);
+    case 3: return launch_fwd<64, 3>(ds, q, k, v, a, total_T, bound, s);
+    case 10: return launch_fwd<128, 0>(ds, q, k, v, a, total_T, bound, s);
+    case 12: return launch_fwd<128, 2>(ds, q, k, v, a, total_T, bound, s);
+    case 13: return launch_fwd<128, 3>(ds, q, k, v, a, total_T, bound, s);
+  }
+  return FA_ERR_UNSUPPORTED;
+}
+
+size_t vec_bytes(int tokens, int Hq) {
+  const size_t b = static_cast<size_t>(Hq) * (static_cast<size_t>(tokens) + fa::kVecSlack) * sizeof(float);
+  return (b + 255) & ~size_t(255);
+}
+
+template <int D>
+fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* dout,
+                       fa::BwdArgs a, long long units_dq, long long units_dkdv, cudaStream_t stream) {
+  constexpr int STAGES = 4;
+  auto kdq = fa::fa_bwd_dq_kernel<D, STAGES>;
+  auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES>;
+  const int smem_dq = static_cast<int>(sizeof(fa::DqSmem<D, STAGES>)) + 1024;
+  const int smem_dkv = static_cast<int>(sizeof(fa::DkvSmem<D, STAGES>)) + 1024;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    bool& done = ds->bwd_attr[D == 128 ? 1 : 0];
+    if (!done) {
+      if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess ||
+          cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv) != cudaSuccess)
+        return FA_ERR_CUDA;
+      done = true;
+    }
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  fa_status_t st;
+  const int T = a.total_T;
+  if ((st = encode_rows(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hq, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hq, D)) != FA_OK) return st;
+  a.timeout_ns = g_timeout_ns.load();
+  a.status = ds->status;
+  // D and LSE in base 2 (one warp per row, 8 warps per block)
+  const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
+  long long pre_blocks = (rows + 7) / 8;
+  if (pre_blocks > static_cast<long long>(ds->sms) * 32) pre_blocks = static_cast<long long>(ds->sms) * 32;
+  fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa::BwdArgs akv = a;
+  akv.num_units = static_cast<int>(units_dkdv);
+  const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
+  if (g1 > 0) kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa::BwdArgs aq = a;
+  aq.num_units = static_cast<int>(units_dq);
+  const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
+  if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                         const int* cu, int nseq, int N, int total_T, int Hq, int Hkv, int d, int causal,
+                         float scale, void* stream) {
+  fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
+  if (st != FA_OK) return st;
+  if (!dout || !dq || !dk || !dv || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  const size_t vb = vec_bytes(total_T, Hq);
+  if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < 2 * vb) return FA_ERR_WORKSPACE;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  fa::BwdArgs a{};
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.lse2 = static_cast<float*>(workspace);
+  a.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) + vb);
+  a.cu_seqlens = cu;
+  a.nseq = nseq;
+  a.N = N;
+  a.total_T = total_T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.lse_head_stride = cu ? total_T : N;
+  a.ws_stride = total_T + fa::kVecSlack;
+  const long long nt = (N + 127) / 128;
+  long long udq, ukv;
+  if (cu == nullptr) {
+    udq = static_cast<long long>(nseq) * Hq * nt;
+    ukv = static_cast<long long>(nseq) * Hkv * nt;
+  } else {
+    const long long by_len = static_cast<long long>(nseq) * nt;
+    const long long by_tok = (static_cast<long long>(total_T) + 127) / 128 + nseq;
+    const long long t = by_len < by_tok ? by_len : by_tok;
+    udq = t * Hq;  // upper bounds; the exact counts are recomputed on the device
+    ukv = t * Hkv;
+  }
+  if (udq > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_bwd<128>(ds, q, k, v, dout, a, udq, ukv, s)
+                  : launch_bwd<64>(ds, q, k, v, dout, a, udq, ukv, s);
 }
 
 }  // namespace
@@ -199,22 +310,32 @@ fa_status_t fa_fwd_fp8(const void*, const void*, const void*, const float*, cons
 }
 
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
-  if (tokens <= 0 || Hq <= 0 || d <= 0 || nseq < 0) return 0;
-  const size_t dq_acc = static_cast<size_t>(tokens) * Hq * d * sizeof(float);
-  const size_t dterm = static_cast<size_t>(tokens) * Hq * sizeof(float);
-  const size_t sems = (static_cast<size_t>(tokens) / 128 + static_cast<size_t>(nseq) + 1) * Hq * sizeof(int);
-  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return up(dq_acc) + up(dterm) + up(sems);
+  (void)nseq;
+  (void)d;
+  if (tokens <= 0 || Hq <= 0) return 0;
+  return 2 * vec_bytes(tokens, Hq);
 }
 
-fa_status_t fa_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
-                   void*, void*, size_t, int, int, int, int, int, int, float, void*) {
-  return FA_ERR_UNSUPPORTED;
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                   void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N,
+                   int d, int causal, float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
+                      causal, scale, stream);
 }
 
-fa_status_t fa_bwd_varlen(const void*, const void*, const void*, const void*, const float*, const void*, void*,
-                          void*, void*, void*, size_t, const int*, int, int, int, int, int, int, int, float, void*) {
-  return FA_ERR_UNSUPPORTED;
+fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                          const int* cu_seqlens, int nseq, int max_seqlen, int total_T, int Hq, int Hkv, int d,
+                          int causal, float scale, void* stream) {
+  if (nseq < 0 || total_T < 0 || max_seqlen < 0 || cu_seqlens == nullptr || !aligned(cu_seqlens, 4))
+    return FA_ERR_INVALID_ARG;
+  if (nseq == 0 || total_T == 0 || max_seqlen == 0) return FA_OK;
+  if (max_seqlen > 131072 || total_T > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total_T,
+                      Hq, Hkv, d, causal, scale, stream);
 }
 
 fa_status_t fa_get_status(void* stream) {
@@ -245,5 +366,11 @@ const char* fa_status_string(fa_status_t s) {
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
 
 void fa_debug_set_inject(int mode) { g_inject.store(mode); }
+
+fa_status_t fa_set_exp_emulation(int pairs_of_8) {
+  if (pairs_of_8 != 0 && pairs_of_8 != 2 && pairs_of_8 != 3) return FA_ERR_UNSUPPORTED;
+  g_exp_emu.store(pairs_of_8);
+  return FA_OK;
+}
 
 }  // extern "C"

@@ -1,0 +1,752 @@
+// Backward pass of exact attention on sm_100a (bf16 in, fp32 accumulation),
+// recomputing the scores from Q, K, V and the forward's LSE instead of storing
+// P (catalogue record "Dao and colleagues: IO-aware exact attention with
+// FlashAttention", summary: tiled operations and recomputation).
+//
+// Gradient of sum(O * dO), per (sequence, query head h, key/value head g):
+//   P = exp(scale * Q K^T - LSE),  D_i = sum_c dO_ic O_ic,
+//   dS = P * (dO V^T - D),  dV = P^T dO,  dK = scale * dS^T Q,  dQ = scale * dS K.
+//
+// Three kernels, deterministic by construction (no atomics, every output
+// element is written once by one CTA):
+//   fa_bwd_pre_kernel   D and LSE*log2(e) per query row into the workspace.
+//   fa_bwd_dkdv_kernel  one CTA per (sequence, kv head, 128-key tile): walks
+//                       the GQA group's query heads and query tiles, keeps
+//                       S^T, dP^T, dV, dK in TMEM (4 x 128 columns).
+//   fa_bwd_dq_kernel    one CTA per (sequence, query head, 128-row tile):
+//                       recomputes S and dP per key block, dQ in TMEM.
+// The dQ kernel recomputes S and dP (three GEMMs per tile pair instead of
+// one), which keeps dQ free of cross-CTA reductions.
+//
+// Elementwise warps: 8 warps, two per TMEM lane quadrant; warp w handles the
+// rows (lanes) 32*(w%4).. and the column half w/4 of each 128-column tile.
+#pragma once
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+
+constexpr int kThreadsBwd = 320;  // 8 elementwise warps, producer, MMA issuer
+constexpr int kVecSlack = 128;    // workspace rows past the last token of each head
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdArgs {
+  const void* o;
+  const void* dout;
+  const float* lse;     // forward LSE (natural log)
+  void* dq;
+  void* dk;
+  void* dv;
+  float* lse2;          // workspace [Hq][total_T + 128]: LSE * log2(e), +inf past the end
+  float* dvec;          // workspace [Hq][total_T + 128]: D, 0 past the end
+  const int* cu_seqlens;
+  int nseq;             // padded: B
+  int N;                // padded: N; varlen: max_seqlen
+  int total_T;
+  int Hq, Hkv;
+  int causal;
+  float scale;
+  float scale_log2;
+  int lse_head_stride;  // forward LSE: padded N, varlen total_T
+  int ws_stride;        // total_T + 128
+  int num_units;
+  uint64_t timeout_ns;
+  int* status;
+};
+
+// ------------------------------------------------------------------ pre
+// One warp per (head, token) row: D = dot(dO, O) in fp32 and LSE in base 2.
+// The 128 slack entries per head hold +inf (LSE) and 0 (D) so that tile
+// loads past a sequence end read harmless values.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  constexpr int PER = D / 32;  // elements per lane
+  for (long long r = w0; r < rows; r += nw) {
+    const int h = static_cast<int>(r / a.ws_stride);
+    const int tok = static_cast<int>(r - static_cast<long long>(h) * a.ws_stride);
+    if (tok >= a.total_T) {
+      if (lane == 0) {
+        a.lse2[r] = INFINITY;
+        a.dvec[r] = 0.f;
+      }
+      continue;
+    }
+    const size_t base = (static_cast<size_t>(tok) * a.Hq + h) * D + lane * PER;
+    const __nv_bfloat16* op = reinterpret_cast<const __nv_bfloat16*>(a.o) + base;
+    const __nv_bfloat16* gp = reinterpret_cast<const __nv_bfloat16*>(a.dout) + base;
+    float acc = 0.f;
+    if constexpr (PER == 4) {
+      const uint2 ov = *reinterpret_cast<const uint2*>(op);
+      const uint2 gv = *reinterpret_cast<const uint2*>(gp);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float2 x = __bfloat1622float2(o2[t]);
+        const float2 y = __bfloat1622float2(g2[t]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    } else {
+      const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(op);
+      const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(gp);
+      const float2 x = __bfloat1622float2(o2);
+      const float2 y = __bfloat1622float2(g2);
+      acc = fmaf(x.x, y.x, x.y * y.y);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      size_t li;
+      if (a.cu_seqlens != nullptr) {
+        li = static_cast<size_t>(h) * a.lse_head_stride + tok;
+      } else {
+        const int b = tok / a.N;
+        li = (static_cast<size_t>(b) * a.Hq + h) * a.lse_head_stride + (tok - b * a.N);
+      }
+      a.lse2[r] = a.lse[li] * kLog2e;
+      a.dvec[r] = acc;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+template <int D, int STAGES>
+struct DqSmem {
+  static constexpr int kTileBytes = kBM * D * 2;
+  alignas(1024) uint8_t q[kTileBytes];
+  alignas(1024) uint8_t dout[kTileBytes];
+  alignas(1024) uint8_t kv[STAGES][kTileBytes];
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[STAGES], kv_empty[STAGES];
+  uint64_t s_full[2], dp_full, ds_ready, acc_final, acc_free;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int level_count[1024];
+};
+
+// A operand taken from TMEM where each elementwise column half stored its
+// bf16 pairs: 16-element K step kk of the first half at column 8*kk, of the
+// second half at column 64 + 8*(kk-4).
+__device__ __forceinline__ uint32_t split_a_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+
+// D(M=128, N=DD) (+)= A(TMEM, 128 x 128 split halves) * B(smem [128 x DD] MN-major)
+template <int DD>
+__device__ __forceinline__ void issue_ts_split(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, DD, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_f16_ts(d_tmem, a_tmem + split_a_col(kk), smem_desc(b_smem + kk * 2048, 16384, 1024, kSwizzle128B), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// D(128 x 128) = A(smem [128 x DD] K-major) * B(smem [128 x DD] K-major)^T
+template <int DD>
+__device__ __forceinline__ void issue_ss_nt(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+  issue_qk<DD>(d_tmem, a_smem, b_smem);
+}
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreadsBwd, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const BwdArgs args) {
+  using Smem = DqSmem<D, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(smem_u32(&sm.q_full), 1);
+    mbar_init(smem_u32(&sm.q_empty), 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&sm.kv_full[s]), 1);
+      mbar_init(smem_u32(&sm.kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.s_full[0]), 1);
+    mbar_init(smem_u32(&sm.s_full[1]), 1);
+    mbar_init(smem_u32(&sm.dp_full), 1);
+    mbar_init(smem_u32(&sm.ds_ready), 8);
+    mbar_init(smem_u32(&sm.acc_final), 1);
+    mbar_init(smem_u32(&sm.acc_free), 8);
+    mbar_init(smem_u32(&sm.drain), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  const int nlevels = (args.N + 127) / 128;
+  const bool varlen = args.cu_seqlens != nullptr;
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  __syncthreads();
+  int num_units = args.num_units;
+  if (varlen)
+    num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 7, args.Hq, kThreadsBwd);
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  // TMEM: S0 [0,128) S1 [128,256) dP [256,384) dQ [384, 384+D)
+  const uint32_t tS0 = tmem, tDP = tmem + 256, tDQ = tmem + 384;
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 7};
+  const volatile int* abort = &sm.abort;
+  const int group = args.Hq / args.Hkv;
+  uint32_t prod_issued = 0, q_issued = 0;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      uint32_t kv_prod = 0, it = 0;
+      bool ok = true;
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
+        const Unit un = decode_unit(sched, u);
+        const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        const int hkv = un.h / group;
+        if (!mbar_wait(smem_u32(&sm.q_empty), (it & 1) ^ 1, abort, args.timeout_ns)) {
+          report_error(args.status, kStatusTimeout, 30);
+          ok = false;
+          break;
+        }
+        const uint32_t qbar = smem_u32(&sm.q_full);
+        mbar_expect_tx(qbar, 2 * Smem::kTileBytes);
+        const int row0 = un.tok0 + un.qb2 * kBM;
+        load_tile<D>(smem_u32(sm.q), &tm_q, qbar, un.h, row0);
+        load_tile<D>(smem_u32(sm.dout), &tm_do, qbar, un.h, row0);
+        q_issued = it + 1;
+        for (int j = 0; j < nblk && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = kv_prod % STAGES;
+            if (!mbar_wait(smem_u32(&sm.kv_empty[slot]), ((kv_prod / STAGES) & 1) ^ 1, abort, args.timeout_ns)) {
+              report_error(args.status, kStatusTimeout, 31);
+              ok = false;
+              break;
+            }
+            const uint32_t bar = smem_u32(&sm.kv_full[slot]);
+            mbar_expect_tx(bar, Smem::kTileBytes);
+            load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
+            ++kv_prod;
+          }
+        }
+      }
+      if (!ok) sm.abort = 1;
+      prod_issued = kv_prod;
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      uint32_t kv_cons = 0, it = 0, dsc = 0, sb_cnt = 0;
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        if (!mbar_wait(smem_u32(bar), parity, abort, args.timeout_ns)) {
+          report_error(args.status, kStatusTimeout, site);
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      (void)sb_cnt;
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
+        const Unit un = decode_unit(sched, u);
+        const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        if (!(ok = wait(&sm.q_full, it & 1, 40))) break;
+        const uint32_t qa = smem_u32(sm.q), doa = smem_u32(sm.dout);
+        // prologue: S(0)
+        uint32_t slotK = kv_cons % STAGES;
+        if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 41))) break;
+        ++kv_cons;
+        issue_ss_nt<D>(tS0, qa, smem_u32(sm.kv[slotK]));
+        tc_commit(smem_u32(&sm.s_full[0]));
+        for (int j = 0; j < nblk; ++j) {
+          const uint32_t slotV = kv_cons % STAGES;
+          if (!(ok = wait(&sm.kv_full[slotV], (kv_cons / STAGES) & 1, 42))) break;
+          ++kv_cons;
+          // dP(j) = dO V_j^T
+          issue_ss_nt<D>(tDP, doa, smem_u32(sm.kv[slotV]));
+          tc_commit(smem_u32(&sm.dp_full));
+          tc_commit(smem_u32(&sm.kv_empty[slotV]));
+          uint32_t slotKn = 0;
+          if (j + 1 < nblk) {
+            slotKn = kv_cons % STAGES;
+            if (!(ok = wait(&sm.kv_full[slotKn], (kv_cons / STAGES) & 1, 43))) break;
+            ++kv_cons;
+            issue_ss_nt<D>(tS0 + ((j + 1) & 1) * 128, qa, smem_u32(sm.kv[slotKn]));
+            tc_commit(smem_u32(&sm.s_full[(j + 1) & 1]));
+          }
+          if (j + 1 == nblk) tc_commit(smem_u32(&sm.q_empty));  // last reads of Q and dO issued
+          // dQ += dS K_j
+          if (!(ok = wait(&sm.ds_ready, dsc & 1, 44))) break;
+          ++dsc;
+          if (j == 0 && !(ok = wait(&sm.acc_free, (it & 1) ^ 1, 45))) break;
+          issue_ts_split<D>(tDQ, tDP, smem_u32(sm.kv[slotK]), j > 0);
+          tc_commit(smem_u32(&sm.kv_empty[slotK]));
+          slotK = slotKn;
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&sm.acc_final));
+      }
+      if (!ok) sm.abort = 1;
+      tc_commit(smem_u32(&sm.drain));
+      mbar_wait(smem_u32(&sm.drain), 0, nullptr, args.timeout_ns);
+    }
+  } else {
+    // ---------------- elementwise warps
+    const int half = warp >> 2;
+    const int quad = warp & 3;
+    const int r_in_tile = quad * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+    const float cl = args.scale_log2;
+    uint32_t sc0 = 0, sc1 = 0, dpc = 0, it = 0;
+    bool ok = true;
+    for (int rnd = 0; ok; ++rnd, ++it) {
+      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (u >= num_units) break;
+      const Unit un = decode_unit(sched, u);
+      const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+      const int row = un.qb2 * kBM + r_in_tile;
+      const bool valid = row < un.n;
+      const size_t wi = static_cast<size_t>(un.h) * args.ws_stride + un.tok0 + row;
+      const float lse2 = valid ? args.lse2[wi] : INFINITY;
+      const float dval = valid ? args.dvec[wi] : 0.f;
+      const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;
+      for (int j = 0; j < nblk; ++j) {
+        const int sb = j & 1;
+        const uint32_t par = sb ? (sc1 & 1) : (sc0 & 1);
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[sb]), par, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 50);
+          break;
+        }
+        if (sb) ++sc1; else ++sc0;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld64(tS0 + sb * 128 + half * 64 + lane_bits, sr);
+        float p[64];
+        const int c0 = j * kBN + half * 64;
+        const bool masked_blk = __any_sync(0xffffffffu, c0 + 63 > limit);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -lse2));
+          p[c] = (masked_blk && c0 + c > limit) ? 0.f : x;
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dp_full), dpc & 1, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 51);
+          break;
+        }
+        ++dpc;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t dr[32];
+          tmem_ld32(tDP + half * 64 + ch * 32 + lane_bits, dr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float a0 = p[ch * 32 + 2 * t] * (__uint_as_float(dr[2 * t]) - dval);
+            const float a1 = p[ch * 32 + 2 * t + 1] * (__uint_as_float(dr[2 * t + 1]) - dval);
+            pk[t] = pack_bf16x2(a0, a1);
+          }
+          tmem_st16(tDP + half * 64 + ch * 16 + lane_bits, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.acc_final), it & 1, abort, args.timeout_ns));
+      if (!ok) {
+        if (lane == 0) report_error(args.status, kStatusTimeout, 52);
+        break;
+      }
+      tc_fence_after();
+      constexpr int HC = D / 2;  // dQ columns per half
+      __nv_bfloat16* qrow = reinterpret_cast<__nv_bfloat16*>(args.dq) +
+                            (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D + half * HC;
+#pragma unroll
+      for (int c = 0; c < HC; c += 32) {
+        uint32_t orr[32];
+        tmem_ld32(tDQ + half * HC + c + lane_bits, orr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          pk[t] = pack_bf16x2(__uint_as_float(orr[2 * t]) * args.scale, __uint_as_float(orr[2 * t + 1]) * args.scale);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(qrow + c);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.acc_free));
+    }
+    if (!ok) sm.abort = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (sm.abort && warp == 8 && lane == 0) {
+    for (uint32_t i = (prod_issued > STAGES ? prod_issued - STAGES : 0); i < prod_issued; ++i)
+      mbar_wait(smem_u32(&sm.kv_full[i % STAGES]), (i / STAGES) & 1, nullptr, args.timeout_ns);
+    if (q_issued > 0) mbar_wait(smem_u32(&sm.q_full), (q_issued - 1) & 1, nullptr, args.timeout_ns);
+  }
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+template <int D, int STAGES>
+struct DkvSmem {
+  static constexpr int kTileBytes = kBM * D * 2;
+  alignas(1024) uint8_t k[kTileBytes];
+  alignas(1024) uint8_t v[kTileBytes];
+  alignas(1024) uint8_t qo[STAGES][kTileBytes];  // Q_i, dO_i alternating
+  float vec[STAGES / 2][2][128];                 // per step: LSE2, D of the 128 query columns
+  uint64_t kv_full, kv_empty;
+  uint64_t qo_full[STAGES], qo_empty[STAGES];
+  uint64_t s_full, dp_full, p_ready, ds_ready, acc_final, acc_free;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int level_count[1024];
+};
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(kThreadsBwd, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdArgs args) {
+  static_assert(STAGES % 2 == 0, "Q and dO alternate in the ring");
+  using Smem = DkvSmem<D, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(smem_u32(&sm.kv_full), 1);
+    mbar_init(smem_u32(&sm.kv_empty), 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&sm.qo_full[s]), 1);
+      mbar_init(smem_u32(&sm.qo_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.dp_full), 1);
+    mbar_init(smem_u32(&sm.p_ready), 8);
+    mbar_init(smem_u32(&sm.ds_ready), 8);
+    mbar_init(smem_u32(&sm.acc_final), 1);
+    mbar_init(smem_u32(&sm.acc_free), 8);
+    mbar_init(smem_u32(&sm.drain), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  const int nlevels = (args.N + 127) / 128;
+  const bool varlen = args.cu_seqlens != nullptr;
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  __syncthreads();
+  int num_units = args.num_units;
+  if (varlen)
+    num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 7, args.Hkv, kThreadsBwd);
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  // TMEM: S^T [0,128) dP^T [128,256) dV [256,256+D) dK [384,384+D)
+  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+  // causal: the heaviest key tiles are the first ones (most query tiles see them)
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hkv, args.causal, nlevels, sm.level_count, 7};
+  const volatile int* abort = &sm.abort;
+  const int group = args.Hq / args.Hkv;
+  uint32_t prod_issued = 0, kv_issued = 0;
+
+  // steps of a unit: (query head of the group, query tile) pairs
+  auto unit_steps = [&](const Unit& un, int& i0, int& nqt) {
+    const int nq = (un.n + 127) / 128;
+    i0 = args.causal ? un.qb2 : 0;
+    nqt = nq - i0;
+    return group * nqt;
+  };
+
+  if (warp == 8) {
+    uint32_t qo_prod = 0, it = 0;
+    bool ok = true;
+    for (int rnd = 0; ok; ++rnd, ++it) {
+      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (u >= num_units) break;
+      const Unit un = decode_unit(sched, u);
+      int i0, nqt;
+      const int nsteps = unit_steps(un, i0, nqt);
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.kv_empty), (it & 1) ^ 1, abort, args.timeout_ns));
+      if (!ok) {
+        if (lane == 0) report_error(args.status, kStatusTimeout, 60);
+        break;
+      }
+      if (lane == 0) {
+        const uint32_t bar = smem_u32(&sm.kv_full);
+        mbar_expect_tx(bar, 2 * Smem::kTileBytes);
+        load_tile<D>(smem_u32(sm.k), &tm_k, bar, un.h, un.tok0 + un.qb2 * kBN);
+        load_tile<D>(smem_u32(sm.v), &tm_v, bar, un.h, un.tok0 + un.qb2 * kBN);
+      }
+      kv_issued = it + 1;
+      for (int st = 0; st < nsteps && ok; ++st) {
+        const int hq = un.h * group + st / nqt;
+        const int qi = i0 + st % nqt;
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t slot = qo_prod % STAGES;
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.qo_empty[slot]), ((qo_prod / STAGES) & 1) ^ 1, abort,
+                                                 args.timeout_ns));
+          if (!ok) {
+            if (lane == 0) report_error(args.status, kStatusTimeout, 61);
+            break;
+          }
+          if (w == 0) {
+            // the query tile's LSE2 and D, 4 each per lane
+            float* vec = sm.vec[(qo_prod / 2) % (STAGES / 2)][0];
+            const size_t wbase = static_cast<size_t>(hq) * args.ws_stride + un.tok0 + qi * kBM;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              vec[lane + 32 * t] = args.lse2[wbase + lane + 32 * t];
+              vec[128 + lane + 32 * t] = args.dvec[wbase + lane + 32 * t];
+            }
+            __syncwarp();
+          }
+          if (lane == 0) {
+            const uint32_t bar = smem_u32(&sm.qo_full[slot]);
+            mbar_expect_tx(bar, Smem::kTileBytes);
+            load_tile<D>(smem_u32(sm.qo[slot]), w == 0 ? &tm_q : &tm_do, bar, hq, un.tok0 + qi * kBM);
+          }
+          ++qo_prod;
+        }
+      }
+    }
+    if (!ok && lane == 0) sm.abort = 1;
+    prod_issued = qo_prod;
+  } else if (warp == 9) {
+    if (lane == 0) {
+      uint32_t qo_cons = 0, it = 0, pc = 0, dsc = 0;
+      bool ok = true;
+      auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
+        if (!mbar_wait(smem_u32(bar), parity, abort, args.timeout_ns)) {
+          report_error(args.status, kStatusTimeout, site);
+          return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
+        const Unit un = decode_unit(sched, u);
+        int i0, nqt;
+        const int nsteps = unit_steps(un, i0, nqt);
+        if (!(ok = wait(&sm.kv_full, it & 1, 70))) break;
+        const uint32_t ka = smem_u32(sm.k), va = smem_u32(sm.v);
+        // prologue: S^T(0), dP^T(0)
+        uint32_t slotQ = qo_cons % STAGES;
+        if (!(ok = wait(&sm.qo_full[slotQ], (qo_cons / STAGES) & 1, 71))) break;
+        uint32_t slotO = (qo_cons + 1) % STAGES;
+        issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[slotQ]));
+        tc_commit(smem_u32(&sm.s_full));
+        if (!(ok = wait(&sm.qo_full[slotO], ((qo_cons + 1) / STAGES) & 1, 72))) break;
+        issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[slotO]));
+        tc_commit(smem_u32(&sm.dp_full));
+        qo_cons += 2;
+        for (int st = 0; st < nsteps; ++st) {
+          const bool has_next = st + 1 < nsteps;
+          // dV += P^T dO
+          if (!(ok = wait(&sm.p_ready, pc & 1, 73))) break;
+          ++pc;
+          if (st == 0 && !(ok = wait(&sm.acc_free, (it & 1) ^ 1, 74))) break;
+          issue_ts_split<D>(tDV, tS, smem_u32(sm.qo[slotO]), st > 0);
+          uint32_t nQ = 0, nO = 0;
+          if (has_next) {
+            nQ = qo_cons % STAGES;
+            nO = (qo_cons + 1) % STAGES;
+            if (!(ok = wait(&sm.qo_full[nQ], (qo_cons / STAGES) & 1, 75))) break;
+            issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[nQ]));
+            tc_commit(smem_u32(&sm.s_full));
+          }
+          // dK += dS^T Q
+          if (!(ok = wait(&sm.ds_ready, dsc & 1, 76))) break;
+          ++dsc;
+          issue_ts_split<D>(tDK, tDP, smem_u32(sm.qo[slotQ]), st > 0);
+          tc_commit(smem_u32(&sm.qo_empty[slotQ]));
+          tc_commit(smem_u32(&sm.qo_empty[slotO]));
+          if (has_next) {
+            if (!(ok = wait(&sm.qo_full[nO], ((qo_cons + 1) / STAGES) & 1, 77))) break;
+            issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[nO]));
+            tc_commit(smem_u32(&sm.dp_full));
+            qo_cons += 2;
+            slotQ = nQ;
+            slotO = nO;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&sm.acc_final));
+        tc_commit(smem_u32(&sm.kv_empty));
+      }
+      if (!ok) sm.abort = 1;
+      tc_commit(smem_u32(&sm.drain));
+      mbar_wait(smem_u32(&sm.drain), 0, nullptr, args.timeout_ns);
+    }
+  } else {
+    // ---------------- elementwise warps: thread = key row, half = query column half
+    const int half = warp >> 2;
+    const int quad = warp & 3;
+    const int r_in_tile = quad * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
+    const float cl = args.scale_log2;
+    uint32_t sc = 0, dpc = 0, it = 0, vstep = 0;
+    bool ok = true;
+    for (int rnd = 0; ok; ++rnd, ++it) {
+      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (u >= num_units) break;
+      const Unit un = decode_unit(sched, u);
+      int i0, nqt;
+      const int nsteps = unit_steps(un, i0, nqt);
+      const int key = un.qb2 * kBN + r_in_tile;  // key row within the sequence
+      const bool valid = key < un.n;
+      for (int st = 0; st < nsteps; ++st, ++vstep) {
+        const int qi = i0 + st % nqt;
+        const float* vec = sm.vec[vstep % (STAGES / 2)][0];
+        const int q0 = qi * kBM + half * 64;  // first query column of this half
+        // the producer stored this step's LSE2/D before arriving on the Q
+        // tile's barrier: waiting on it makes those stores visible here
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.qo_full[(2 * vstep) % STAGES]),
+                                               ((2 * vstep) / STAGES) & 1, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 83);
+          break;
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full), sc & 1, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 80);
+          break;
+        }
+        ++sc;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld64(tS + half * 64 + lane_bits, sr);
+        // a query column q is hidden from key k when q >= n or (causal and k > q)
+        const int lo = args.causal ? key : 0;  // smallest visible query
+        const bool masked_blk = __any_sync(0xffffffffu, q0 < lo || q0 + 63 >= un.n);
+        float p[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -vec[half * 64 + c]));
+          p[c] = (masked_blk && (q0 + c < lo || q0 + c >= un.n)) ? 0.f : x;
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(p[2 * t], p[2 * t + 1]);
+          tmem_st32(tS + half * 64 + lane_bits, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_ready));
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dp_full), dpc & 1, abort, args.timeout_ns));
+        if (!ok) {
+          if (lane == 0) report_error(args.status, kStatusTimeout, 81);
+          break;
+        }
+        ++dpc;
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t dr[32];
+          tmem_ld32(tDP + half * 64 + ch * 32 + lane_bits, dr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int c = ch * 32 + 2 * t;
+            const float a0 = p[c] * (__uint_as_float(dr[2 * t]) - vec[128 + half * 64 + c]);
+            const float a1 = p[c + 1] * (__uint_as_float(dr[2 * t + 1]) - vec[128 + half * 64 + c + 1]);
+            pk[t] = pack_bf16x2(a0, a1);
+          }
+          tmem_st16(tDP + half * 64 + ch * 16 + lane_bits, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.ds_ready));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.acc_final), it & 1, abort, args.timeout_ns));
+      if (!ok) {
+        if (lane == 0) report_error(args.status, kStatusTimeout, 82);
+        break;
+      }
+      tc_fence_after();
+      constexpr int HC = D / 2;
+      const size_t rowoff = (static_cast<size_t>(un.tok0 + key) * args.Hkv + un.h) * D + half * HC;
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst_row = reinterpret_cast<__nv_bfloat16*>(which == 0 ? args.dv : args.dk) + rowoff;
+        const uint32_t src = (which == 0 ? tDV : tDK) + half * HC + lane_bits;
+        const float mul = which == 0 ? 1.f : args.scale;
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t orr[32];
+          tmem_ld32(src + c, orr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            pk[t] = pack_bf16x2(__uint_as_float(orr[2 * t]) * mul, __uint_as_float(orr[2 * t + 1]) * mul);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.acc_free));
+    }
+    if (!ok) sm.abort = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (sm.abort && warp == 8 && lane == 0) {
+    for (uint32_t i = (prod_issued > STAGES ? prod_issued - STAGES : 0); i < prod_issued; ++i)
+      mbar_wait(smem_u32(&sm.qo_full[i % STAGES]), (i / STAGES) & 1, nullptr, args.timeout_ns);
+    if (kv_issued > 0) mbar_wait(smem_u32(&sm.kv_full), (kv_issued - 1) & 1, nullptr, args.timeout_ns);
+  }
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -94,7 +94,40 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
 }
 
-template <int D, int STAGES>
+// Exponentials of one 128-column row slice, packed to bf16 pairs and stored
+// over the first 64 TMEM columns of the S tile; returns the fp32 row sum.
+// Scale and sum run on packed fp32 pairs; EMU of every 8 pairs take exp2 on
+// the FMA pipe (exp2_poly_pair), the rest on MUFU.
+template <int EMU>
+__device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, float cl, float mc) {
+  const uint64_t c2 = f2(cl, cl);
+  const uint64_t nmc2 = f2(-mc, -mc);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const int e = c4 * 32 + 2 * t;
+      const uint64_t x2 = f2_fma(f2(s[e], s[e + 1]), c2, nmc2);
+      float p0, p1;
+      if ((t & 7) < EMU) {
+        exp2_poly_pair(x2, p0, p1);
+      } else {
+        const float2 x = f2_split(x2);
+        p0 = ex2_approx(x.x);
+        p1 = ex2_approx(x.y);
+      }
+      acc[t & 3] = f2_add(acc[t & 3], f2(p0, p1));
+      pk[t] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(S + c4 * 16, pk);
+  }
+  const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
+  return a.x + a.y;
+}
+
+template <int D, int STAGES, int EMU>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -125,9 +158,6 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   }
   const int nlevels = (args.N + 255) / 256;
   const bool varlen = args.cu_seqlens != nullptr;
-  if (varlen) {
-    for (int L = tid; L < nlevels; L += kThreadsFwd) sm.level_count[L] = 0;
-  }
   if (warp == 9) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
@@ -139,20 +169,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   }
   __syncthreads();
   int num_units = args.num_units;
-  if (varlen) {
-    for (int s = tid; s < args.nseq; s += kThreadsFwd) {
-      const int n = __ldg(args.cu_seqlens + s + 1) - __ldg(args.cu_seqlens + s);
-      const int nl = min((n + 255) >> 8, nlevels);
-      for (int L = 0; L < nl; ++L) atomicAdd(&sm.level_count[L], 1);
-    }
-    __syncthreads();
-    int tot = 0;
-    for (int L = 0; L < nlevels; ++L) tot += sm.level_count[L];
-    num_units = tot * args.Hq;
-  }
+  if (varlen)
+    num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 8, args.Hq, kThreadsFwd);
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, args.causal, nlevels, sm.level_count};
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 8};
   const volatile int* abort = &sm.abort;
   const int group = args.Hq / args.Hkv;
   uint32_t prod_issued = 0;  // K/V loads issued by the producer thread
@@ -163,7 +184,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     if (lane == 0) {
       uint32_t kv_prod = 0, it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
         const int nblk = num_kv_blocks(un, args.causal);
         const int hkv = un.h / group;
@@ -214,7 +237,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         tc_fence_after();
         return true;
       };
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
         const int nblk = num_kv_blocks(un, args.causal);
         if (!(ok = wait(&sm.q_full, it & 1, 10))) break;
@@ -282,7 +307,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const float cl = args.scale_log2;
     uint32_t sc = 0, it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++it) {
+    for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
       const int nblk = num_kv_blocks(un, args.causal);
       const int row = un.qb2 * 2 * kBM + tile * kBM + r_in_tile;  // row within the sequence
@@ -299,20 +326,27 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         ++sc;
         tc_fence_after();
         uint32_t sr[128];
-        tmem_ld32(S + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(S + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(S + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld128(S, sr);
         float* s = reinterpret_cast<float*>(sr);
         const int kv0 = j * kBN;
-        if (kv0 + kBN - 1 > limit) {
+        // Warp-uniform: the exponential path below holds warp-collective
+        // TMEM stores, so every lane of a warp must take the same branch.
+        const bool masked_blk = __any_sync(0xffffffffu, kv0 + kBN - 1 > limit);
+        if (masked_blk) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (kv0 + c > limit) s[c] = -INFINITY;
         }
-        float mt = s[0];
+        // row maximum: four independent chains of three-input max
+        float mx[4];
 #pragma unroll
-        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float a = fmax3(s[q4 * 32 + 0], s[q4 * 32 + 1], s[q4 * 32 + 2]);
+#pragma unroll
+          for (int c = 3; c + 1 < 32; c += 2) a = fmax3(a, s[q4 * 32 + c], s[q4 * 32 + c + 1]);
+          mx[q4] = fmaxf(a, s[q4 * 32 + 31]);
+        }
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         const bool need = (mt - m) * cl > kTau;
         const float m_new = need ? mt : m;
         const float alpha = need ? ex2_approx((m - m_new) * cl) : 1.f;
@@ -329,20 +363,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             tmem_st32(O + c, orr);
           }
         }
-        const float mc = m_new * cl;
-        float lsum = 0.f;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const float p0 = ex2_approx(fmaf(s[c4 * 32 + 2 * t], cl, -mc));
-            const float p1 = ex2_approx(fmaf(s[c4 * 32 + 2 * t + 1], cl, -mc));
-            lsum += p0 + p1;
-            pk[t] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(S + c4 * 16, pk);
-        }
+        // P = 2^(s*c - m*c), written as bf16 over the first 64 columns of S
+        const float lsum = masked_blk ? softmax_exp_store<0>(s, S, cl, m_new * cl)
+                                      : softmax_exp_store<EMU>(s, S, cl, m_new * cl);
         l = l * alpha + lsum;
         m = m_new;
         tmem_st_wait();

@@ -210,6 +210,40 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 #undef FA_R8
+
+// Four 32-column loads of 32x32b shape (128 consecutive columns) and a single
+// wait: one TMEM round trip for a whole 128-column row slice.
+#define FA_O8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
+                 "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,"
+      "%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : FA_O8(0), FA_O8(8), FA_O8(16), FA_O8(24), FA_O8(32), FA_O8(40), FA_O8(48), FA_O8(56), FA_O8(64),
+        FA_O8(72), FA_O8(80), FA_O8(88), FA_O8(96), FA_O8(104), FA_O8(112), FA_O8(120)
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+}
+// Two 32-column loads (64 consecutive columns) and one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : FA_O8(0), FA_O8(8), FA_O8(16), FA_O8(24), FA_O8(32), FA_O8(40), FA_O8(48), FA_O8(56)
+      : "r"(taddr), "r"(taddr + 32)
+      : "memory");
+}
+#undef FA_O8
 #define FA_S8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
                  "r"(r[i + 6]), "r"(r[i + 7])
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -231,12 +265,83 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Per-warpgroup register reallocation (all four warps of the warpgroup
+// execute it). The sum over warpgroups must stay within the registers the
+// block was launched with.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// three-input maximum (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// packed fp32 pairs (sm_100 f32x2 arithmetic): element 0 in the low half
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// 2^x for a pair of floats on the FMA/ALU pipes instead of MUFU (x <= 127).
+// Method: Cody-Waite style split x = n + f with n = round(x) obtained by the
+// round-to-nearest addition of 1.5*2^23, f in [-0.5, 0.5]; 2^f by a cubic
+// fitted to 2^f on [-0.5, 0.5] (iteratively reweighted least squares in the
+// relative sense, max relative error 7.5e-5); 2^n added to the exponent field
+// as an integer. Inputs below -125 are clamped to -125 (2^-125 ~ 2.4e-38), so
+// the result is never denormal or wrapped.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& r0, float& r1) {
+  float2 x = f2_split(x2);
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const uint64_t xc = f2(x.x, x.y);
+  const uint64_t magic = f2(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(xc, magic);
+  const uint64_t n = f2_add(t, f2(-12582912.f, -12582912.f));
+  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(fr, f2(0.05517132207751274f, 0.05517132207751274f),
+                      f2(0.24261054396629333f, 0.24261054396629333f));
+  p = f2_fma(p, fr, f2(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, fr, f2(0.9999281167984009f, 0.9999281167984009f));
+  const float2 pv = f2_split(p);
+  const float2 tv = f2_split(t);
+  r0 = __uint_as_float(__float_as_uint(pv.x) + (__float_as_uint(tv.x) << 23));
+  r1 = __uint_as_float(__float_as_uint(pv.y) + (__float_as_uint(tv.y) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
