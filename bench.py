@@ -254,31 +254,34 @@ def run_ours(args):
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error during warm-up")
 
-    # timed region: K steps, L2 flushed before each (outside the step's events)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # timed region: K steps, L2 flushed before each (outside the step's events).
+    # The backward runs as its three parts back to back (exactly fa_bwd's
+    # work) with events between them, for the per-kernel roofline.
+    nev = 5 if with_bwd else 2
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
-            a, mid, b = ev[i]
-            a.record(stream)
+            e = ev[i]
+            e[0].record(stream)
             fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
-            mid.record(stream)
+            e[1].record(stream)
             if with_bwd:
-                fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, int(causal), scale, sptr)
-            b.record(stream)
+                for j, part in enumerate((fa.FA_BWD_PREPARE, fa.FA_BWD_DKDV, fa.FA_BWD_DQ)):
+                    fa.fa_bwd_part(part, q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d,
+                                   int(causal), scale, sptr)
+                    e[2 + j].record(stream)
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     st = fa.fa_get_status(sptr)
     if st != fa.FA_OK:
         raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
-    step_ms = [a.elapsed_time(b) for a, _, b in ev]
-    fwd_ms = [a.elapsed_time(m) for a, m, _ in ev]
-    bwd_ms = [m.elapsed_time(b) for _, m, b in ev]
+    step_ms = [e[0].elapsed_time(e[-1]) for e in ev]
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(nev - 1)]
     tot_ms = sum(step_ms)
     if pg:
         t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
@@ -289,19 +292,37 @@ def run_ours(args):
     f_step = f_fwd * (3.5 if with_bwd else 1.0)
     value = f_step * world * args.steps / (tot_ms * 1e-3) / 1e12
 
-    # roofline of the dominant kernel (largest share of the step)
+    # roofline of the dominant kernel (largest share of the step). Flops per
+    # launch are the tensor-core flops the kernel executes: forward 2 GEMMs
+    # (= the algorithmic forward count), dK/dV 4 GEMMs, dQ 3 GEMMs (S and dP
+    # recomputed); the D/LSE preparation is HBM-bound (bytes moved).
     pk = peaks()
-    fwd_avg = sum(fwd_ms) / len(fwd_ms)
-    bwd_avg = sum(bwd_ms) / len(bwd_ms) if with_bwd else 0.0
-    if with_bwd and bwd_avg > fwd_avg:
-        dom, dom_flops, dom_ms = "fa_bwd", 2.5 * f_fwd, bwd_avg
+    avg = [sum(x) / len(x) for x in seg]
+    tok = B * N
+    kernels = [{"kernel": "fa_fwd_sm100_kernel", "ms": avg[0], "bound": "tensor", "flops": f_fwd}]
+    if with_bwd:
+        pre_bytes = 2 * tok * Hq * d * 2 + tok * Hq * 4 + 2 * Hq * (tok + 128) * 4
+        kernels += [{"kernel": "fa_bwd_pre_kernel", "ms": avg[1], "bound": "hbm", "bytes": pre_bytes},
+                    {"kernel": "fa_bwd_dkdv_kernel", "ms": avg[2], "bound": "tensor", "flops": 2.0 * f_fwd},
+                    {"kernel": "fa_bwd_dq_kernel", "ms": avg[3], "bound": "tensor", "flops": 1.5 * f_fwd}]
+    for kk in kernels:
+        if kk["bound"] == "tensor":
+            kk["achieved_tflops"] = kk["flops"] / (kk["ms"] * 1e-3) / 1e12
+            kk["frac"] = kk["achieved_tflops"] / pk["bf16_tflops"]
+        else:
+            kk["achieved_gbs"] = kk["bytes"] / (kk["ms"] * 1e-3) / 1e9
+            kk["frac"] = kk["achieved_gbs"] / pk["hbm_gbs"]
+    dom = max(kernels, key=lambda x: x["ms"])
+    if dom["bound"] == "tensor":
+        roofline = {"bound": "tensor", "kernel": dom["kernel"], "achieved": dom["achieved_tflops"],
+                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": dom["frac"],
+                    "traffic": traffic_for(dom["kernel"]),
+                    "peak_source": f"{pk['source']} bf16 burst (cuBLAS)", "kernels": kernels}
     else:
-        dom, dom_flops, dom_ms = "fa_fwd_sm100_kernel", f_fwd, fwd_avg
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": traffic_for(dom),
-                "peak_source": f"{pk['source']} bf16 burst (cuBLAS)",
-                "fwd_ms": fwd_avg, "bwd_ms": bwd_avg if with_bwd else None}
+        roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved_gbs"],
+                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dom["frac"],
+                    "traffic": traffic_for(dom["kernel"]), "peak_source": f"{pk['source']} HBM copy",
+                    "kernels": kernels}
 
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None

@@ -117,6 +117,20 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
                    const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq,
                    int Hkv, int N, int d, int causal, float scale, void* stream);
 
+/*
+ * The backward pass of fa_bwd in separately launchable parts (bit mask):
+ *   FA_BWD_PREPARE  D = dot(dO, O) and the base-2 LSE into the workspace;
+ *   FA_BWD_DKDV     dK and dV (reads the workspace written by PREPARE);
+ *   FA_BWD_DQ       dQ (reads the workspace written by PREPARE).
+ * fa_bwd(...) is fa_bwd_part(FA_BWD_ALL, ...). After PREPARE has completed,
+ * DKDV and DQ are independent and may run concurrently on two streams.
+ * Arguments as fa_bwd; parts outside 1..7 return FA_ERR_INVALID_ARG.
+ */
+enum { FA_BWD_PREPARE = 1, FA_BWD_DKDV = 2, FA_BWD_DQ = 4, FA_BWD_ALL = 7 };
+fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                        int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
+
 /* Backward pass, packed variable-length batch; layouts as fa_fwd_varlen. */
 fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,

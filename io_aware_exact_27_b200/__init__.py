@@ -43,6 +43,7 @@ _SIGS = {
     "fa_bwd_varlen": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_get_status": [_P],
     "fa_set_exp_emulation": [_I],
+    "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
 for _name, _args in _SIGS.items():
     getattr(_lib, _name).argtypes = _args
@@ -59,6 +60,7 @@ _lib.fa_last_device_error_word.argtypes = []
 _lib.fa_last_device_error_word.restype = _I
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_BWD_PREPARE, FA_BWD_DKDV, FA_BWD_DQ, FA_BWD_ALL = 1, 2, 4, 7
 
 
 class FAError(RuntimeError):
@@ -118,6 +120,13 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N
     _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                        _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)),
            "fa_bwd")
+
+
+def fa_bwd_part(parts, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N, d, causal, scale,
+                stream=None):
+    _check(_lib.fa_bwd_part(int(parts), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                            _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal),
+                            float(scale), _stream(stream)), "fa_bwd_part")
 
 
 def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total_T,

@@ -187,7 +187,7 @@ size_t vec_bytes(int tokens, int Hq) {
 
 template <int D>
 fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* dout,
-                       fa::BwdArgs a, long long units_dq, long long units_dkdv, cudaStream_t stream) {
+                       fa::BwdArgs a, long long units_dq, long long units_dkdv, int parts, cudaStream_t stream) {
   constexpr int STAGES = 4;
   auto kdq = fa::fa_bwd_dq_kernel<D, STAGES>;
   auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES>;
@@ -216,24 +216,31 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
   long long pre_blocks = (rows + 7) / 8;
   if (pre_blocks > static_cast<long long>(ds->sms) * 32) pre_blocks = static_cast<long long>(ds->sms) * 32;
-  fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  fa::BwdArgs akv = a;
-  akv.num_units = static_cast<int>(units_dkdv);
-  const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
-  if (g1 > 0) kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  fa::BwdArgs aq = a;
-  aq.num_units = static_cast<int>(units_dq);
-  const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
-  if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (parts & FA_BWD_PREPARE) {
+    fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (parts & FA_BWD_DKDV) {
+    fa::BwdArgs akv = a;
+    akv.num_units = static_cast<int>(units_dkdv);
+    const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
+    if (g1 > 0) kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (parts & FA_BWD_DQ) {
+    fa::BwdArgs aq = a;
+    aq.num_units = static_cast<int>(units_dq);
+    const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
+    if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                          const int* cu, int nseq, int N, int total_T, int Hq, int Hkv, int d, int causal,
-                         float scale, void* stream) {
+                         float scale, void* stream, int parts = FA_BWD_ALL) {
   fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
   if (st != FA_OK) return st;
   if (!dout || !dq || !dk || !dv || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
@@ -278,8 +285,9 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   }
   if (udq > INT32_MAX) return FA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_bwd<128>(ds, q, k, v, dout, a, udq, ukv, s)
-                  : launch_bwd<64>(ds, q, k, v, dout, a, udq, ukv, s);
+  if (parts <= 0 || parts > FA_BWD_ALL) return FA_ERR_INVALID_ARG;
+  return d == 128 ? launch_bwd<128>(ds, q, k, v, dout, a, udq, ukv, parts, s)
+                  : launch_bwd<64>(ds, q, k, v, dout, a, udq, ukv, parts, s);
 }
 
 }  // namespace
@@ -324,6 +332,16 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
   if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
   return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
                       causal, scale, stream);
+}
+
+fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                        int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
+                      causal, scale, stream, parts);
 }
 
 fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
