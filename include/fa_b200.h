@@ -131,6 +131,32 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
                         const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
                         int Hq, int Hkv, int N, int d, int causal, float scale, void* stream);
 
+/*
+ * Backward pass without any device allocation, for callers that cannot
+ * allocate device memory themselves: runtimes that plan all device memory
+ * ahead of time and forbid further allocations while they run, plugins that
+ * have no access to their host's allocator, and code whose memory budget is
+ * fixed once at start-up. (No counterpart in the pages: this is a library
+ * convenience.)
+ *   Arguments and results as fa_bwd, minus the workspace: the scratch lives in
+ *   an 8 MiB array inside the library, on every device that loads it, for the
+ *   life of the process. The problem must fit it:
+ *   fa_bwd_workspace_size(B*N, B, Hq, d) <= 8 MiB, i.e. Hq * (B*N + 128) up
+ *   to about 1.04 million; larger problems return FA_ERR_WORKSPACE and launch
+ *   nothing.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Every call uses the same array: calls whose work overlaps on the GPU (on
+ *   different streams, or from different threads) race on it and must be
+ *   serialised by the caller. The array keeps whatever the last call left;
+ *   nothing in it needs clearing between calls.
+ *   No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                           int causal, float scale, void* stream);
+
 /* Backward pass, packed variable-length batch; layouts as fa_fwd_varlen. */
 fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,

@@ -290,6 +290,30 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
                   : launch_bwd<64>(ds, q, k, v, dout, a, udq, ukv, parts, s);
 }
 
+// ---------------------------------------------------------------- no-allocation backward
+// Scratch of fa_bwd_noalloc: a fixed array in device memory, created when the
+// library is loaded and held by every GPU that loads it until the process
+// exits. Host code must not use the symbol itself as an address (on the host
+// it only names the array); its device address is looked up per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device; looked up once
+// per device (with that device current) and cached.
+fa_status_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -354,6 +378,23 @@ fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const voi
   if (max_seqlen > 131072 || total_T > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
   return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total_T,
                       Hq, Hkv, d, causal, scale, stream);
+}
+
+fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                           int causal, float scale, void* stream) {
+  if (B < 0 || N < 0 || Hq <= 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  // the whole working set must fit the built-in array
+  if (fa_bwd_workspace_size(B * N, B, Hq, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const fa_status_t st = noalloc_scratch_address(&scratch);
+  if (st != FA_OK) return st;
+  // Nothing in the scratch has to start at zero: the first kernel of the
+  // backward writes every entry the later two read.
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, causal, scale,
+                stream);
 }
 
 fa_status_t fa_get_status(void* stream) {
