@@ -87,6 +87,10 @@ fa_status_t fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, 
  *   the value of element x of rows 128*i .. 128*i+127 of head h is code * scale[b,h,i].
  *   o [B,N,Hq,d] bf16, lse [B,Hq,N] float32 (out), as fa_fwd on the dequantised values.
  *   d must be 128.
+ * S = Q K^T runs on e4m3 tensor cores (kind::f8f6f4) with the query and key
+ * block scales folded into the exponent; for O += P V the e4m3 V tiles are
+ * widened to f16 on chip (exactly) and P is rounded to f16 with the V block
+ * scale folded in, so P keeps 11 significant bits instead of e4m3's 4.
  */
 fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
                        const float* k_scale, const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv,
@@ -193,7 +197,8 @@ void fa_set_wait_timeout_ns(uint64_t ns);
 void fa_debug_set_inject(int mode);
 
 /*
- * Tuning knob of the bf16 forward kernels: of every 8 pairs of score
+ * Tuning knob of the bf16 forward kernels (the fp8 forward always uses
+ * MUFU): of every 8 pairs of score
  * elements, how many take their exponential on the FMA pipe (a cubic
  * polynomial after exact range reduction, relative error < 1e-4) instead of
  * the MUFU unit, which otherwise limits the softmax. Accepted: 0, 2, 3

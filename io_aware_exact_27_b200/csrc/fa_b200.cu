@@ -32,7 +32,7 @@ struct DeviceState {
   int sms = 0;
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
-  bool fwd_attr[2][5] = {};
+  bool fwd_attr[3][5] = {};
   bool bwd_attr[2] = {false, false};
 };
 DeviceState g_dev[kMaxDevices];
@@ -105,16 +105,16 @@ fa_status_t check_common(const void* q, const void* k, const void* v, const void
   return FA_OK;
 }
 
-template <int D, int EMU>
+template <int D, int EMU, bool F8 = false>
 fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, fa::FwdArgs a, int tokens,
                        long long units_bound, cudaStream_t stream) {
-  constexpr int STAGES = 4;
-  using Smem = fa::FwdSmem<D, STAGES>;
-  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU>;
+  constexpr int STAGES = F8 ? 6 : 4;
+  using Smem = fa::FwdSmem<D, STAGES, F8>;
+  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU, F8>;
   const int smem = static_cast<int>(sizeof(Smem)) + 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->fwd_attr[D == 128 ? 1 : 0][EMU];
+    bool& done = ds->fwd_attr[F8 ? 2 : (D == 128 ? 1 : 0)][EMU];
     if (!done) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -123,15 +123,17 @@ fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void
   }
   CUtensorMap tq, tk, tv;
   fa_status_t st;
-  if ((st = encode_rows(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hq, D)) != FA_OK) return st;
-  if ((st = encode_rows(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
-  if ((st = encode_rows(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  const CUtensorMapDataType dt = F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  constexpr int EB = F8 ? 1 : 2;
+  if ((st = encode_rows(&tq, q, dt, EB, tokens, a.Hq, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tk, k, dt, EB, tokens, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tv, v, dt, EB, tokens, a.Hkv, D)) != FA_OK) return st;
   a.timeout_ns = g_timeout_ns.load();
   a.inject = g_inject.load();
   a.status = ds->status;
   const int grid = static_cast<int>(units_bound < ds->sms ? units_bound : ds->sms);
   if (grid <= 0) return FA_OK;
-  kern<<<grid, fa::kThreadsFwd, smem, stream>>>(tq, tk, tv, a);
+  kern<<<grid, F8 ? fa::kThreadsFwdF8 : fa::kThreadsFwd, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -336,9 +338,42 @@ fa_status_t fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, 
   return fwd_dispatch(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total_T, Hq, Hkv, d, causal, scale, stream);
 }
 
-fa_status_t fa_fwd_fp8(const void*, const void*, const void*, const float*, const float*, const float*, void*,
-                       float*, int, int, int, int, int, int, float, void*) {
-  return FA_ERR_UNSUPPORTED;
+fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                       const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
+                       float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  fa_status_t st = check_common(q8, k8, v8, o, lse, Hq, Hkv, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q_scale || !k_scale || !v_scale || !aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+    return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  fa::FwdArgs a{};
+  a.o = o;
+  a.lse = lse;
+  a.cu_seqlens = nullptr;
+  a.nseq = B;
+  a.N = N;
+  a.total_T = B * N;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.causal = causal;
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.lse_head_stride = N;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.nblk_s = (N + 127) / 128;
+  const long long bound = static_cast<long long>(B) * Hq * ((N + 255) / 256);
+  if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  a.num_units = static_cast<int>(bound);
+  // exponentials on MUFU only: the FMA pipe is shared with the V widening warps
+  return launch_fwd<128, 0, true>(ds, q8, k8, v8, a, B * N, bound, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {

@@ -1,4 +1,6 @@
-// Forward pass of exact attention on sm_100a (bf16 in, fp32 accumulation).
+// Forward pass of exact attention on sm_100a: bf16 in, or fp8-e4m3 in with
+// per-(head, 128-row block) scales (FA-3 summary, contribution 3: FP8 GEMMs);
+// fp32 accumulation in both.
 //
 // What it computes: O = softmax(scale * Q K^T + mask) V and the per-row
 // natural-log LSE, tile by tile, the score matrix living only in tensor
@@ -25,7 +27,10 @@ namespace fa {
 constexpr int kBM = 128;      // query rows per tile
 constexpr int kBN = 128;      // keys per block
 constexpr int kThreadsFwd = 320;
+// fp8 adds two warps that widen each e4m3 V tile to f16 for the PV MMA
+constexpr int kThreadsFwdF8 = 384;
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, base-2 exponent units
+
 
 struct FwdArgs {
   void* o;
@@ -43,49 +48,91 @@ struct FwdArgs {
   uint64_t timeout_ns;
   int* status;
   int inject;      // test hook: 1 = the producer never loads the first K tile
+  // fp8 only: block scales [B, H, nblk_s] (value = code * scale)
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
+  int nblk_s;
 };
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool F8 = false>
 struct FwdSmem {
-  static constexpr int kTileBytes = kBM * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kTileBytes = kBM * D * (F8 ? 1 : 2);  // one 128 x D tile
   alignas(1024) uint8_t q[2][kTileBytes];
   alignas(1024) uint8_t kv[STAGES][kTileBytes];
+  // fp8: V tiles widened to f16 (exact), double-buffered
+  static constexpr int kV16Bytes = F8 ? kBM * D * 2 : 1024;
+  alignas(1024) uint8_t v16[2][kV16Bytes];
   uint64_t q_full, q_empty;
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+  uint64_t v16_full[2], v16_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   int level_count[512];
 };
 
-// Loads one 128 x D bf16 tile as D/64 boxes of 128 rows x 128 bytes (SW128).
-template <int D>
+// Loads one 128 x D tile (EB bytes per element) as D*EB/128 boxes of 128
+// rows x 128 bytes (SW128).
+template <int D, int EB = 2>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m, uint32_t bar, int head, int row0) {
 #pragma unroll
-  for (int b = 0; b < D / 64; ++b) tma_load_3d(dst + b * 16384, m, bar, b * 64, head, row0);
+  for (int b = 0; b < D * EB / 128; ++b) tma_load_3d(dst + b * 16384, m, bar, b * (128 / EB), head, row0);
 }
 
-template <int D>
+// S = Q K^T over d: each MMA consumes 32 bytes of every row (16 bf16 or 32
+// e4m3 elements), advancing inside the 128-byte swizzle row.
+template <int D, bool F8 = false>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, false);
+  constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(kBM, kBN, false, false) : idesc_bf16_f32(kBM, kBN, false, false);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < D * (F8 ? 1 : 2) / 32; ++kk) {
     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    mma_f16_ss(s_tmem, smem_desc(q_smem + off, 16, 1024, kSwizzle128B),
-               smem_desc(k_smem + off, 16, 1024, kSwizzle128B), idesc, kk > 0 ? 1u : 0u);
+    const uint64_t a = smem_desc(q_smem + off, 16, 1024, kSwizzle128B);
+    const uint64_t b = smem_desc(k_smem + off, 16, 1024, kSwizzle128B);
+    if constexpr (F8)
+      mma_f8_ss(s_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    else
+      mma_f16_ss(s_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-template <int D>
+// O += P V: P (bf16 or f16 pairs) read from TMEM, V a [keys, D] tile (D
+// contiguous) in shared memory as the MN-major B operand: LBO = next 64
+// columns of D (next 16 KB box), SBO = next 8 keys. One MMA covers 16 keys.
+template <int D, bool F16 = false>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, false, true);
+  constexpr uint32_t idesc = F16 ? idesc_f16_f32(kBM, D, false, true) : idesc_bf16_f32(kBM, D, false, true);
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk) {
-    // V tile is [keys, D] (D contiguous): MN-major B operand; LBO = next 64
-    // columns of D (next TMA box), SBO = next 8 keys.
+  for (int kk = 0; kk < kBN / 16; ++kk)
     mma_f16_ts(o_tmem, p_tmem + kk * 8, smem_desc(v_smem + kk * 2048, 16384, 1024, kSwizzle128B), idesc,
                (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// fp8: widens `nkeys` rows (keys) of an e4m3 V tile to f16 (exactly) in the
+// 128B-swizzled MN-major layout the PV MMA reads; thread t of nthreads takes
+// every nthreads-th (key, 16-element chunk). `src` and `dst` point at the
+// first row handled (a multiple of 8 rows into the tile).
+template <int D>
+__device__ __forceinline__ void widen_v_tile(const uint8_t* src, uint8_t* dst, int t, int nthreads, int nkeys) {
+  static_assert(D == 128, "fp8 path is built for d = 128");
+  for (int u = t; u < nkeys * 8; u += nthreads) {
+    const int r = u >> 3;      // key
+    const int c16 = u & 7;     // 16-element (16-byte) chunk of the e4m3 row
+    const uint4 v = *reinterpret_cast<const uint4*>(src + r * 128 + ((c16 ^ (r & 7)) << 4));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h[2 * i] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] & 0xffffu));
+      h[2 * i + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[i] >> 16));
+    }
+    // elements 16*c16 .. +15 -> f16 box c16/4, 8-element chunks 2*(c16%4), +1
+    uint8_t* box = dst + (c16 >> 2) * 16384 + r * 128;
+    const int c8 = 2 * (c16 & 3);
+    *reinterpret_cast<uint4*>(box + ((c8 ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(box + (((c8 + 1) ^ (r & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
   }
 }
 
@@ -94,14 +141,15 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
 }
 
-// Exponentials of one 128-column row slice, packed to bf16 pairs and stored
-// over the first 64 TMEM columns of the S tile; returns the fp32 row sum.
-// Scale and sum run on packed fp32 pairs; EMU of every 8 pairs take exp2 on
-// the FMA pipe (exp2_poly_pair), the rest on MUFU.
-template <int EMU>
-__device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, float cl, float mc) {
-  const uint64_t c2 = f2(cl, cl);
-  const uint64_t nmc2 = f2(-mc, -mc);
+// Exponentials of one 128-column row slice: p = 2^(s*cj - m) in fp32 (the
+// row sum), stored over the first 64 TMEM columns of the S tile as the A
+// operand of the PV MMA: bf16 pairs, or (fp8 path) f16 pairs of p*pmul, the
+// V block scale folded in. Scale and sum run on packed fp32 pairs; EMU of
+// every 8 pairs take exp2 on the FMA pipe (exp2_poly_pair), the rest on MUFU.
+template <int EMU, bool F16>
+__device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, float cj, float m, float pmul) {
+  const uint64_t c2 = f2(cj, cj);
+  const uint64_t nm2 = f2(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
   for (int c4 = 0; c4 < 4; ++c4) {
@@ -109,7 +157,7 @@ __device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, f
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
       const int e = c4 * 32 + 2 * t;
-      const uint64_t x2 = f2_fma(f2(s[e], s[e + 1]), c2, nmc2);
+      const uint64_t x2 = f2_fma(f2(s[e], s[e + 1]), c2, nm2);
       float p0, p1;
       if ((t & 7) < EMU) {
         exp2_poly_pair(x2, p0, p1);
@@ -119,7 +167,10 @@ __device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, f
         p1 = ex2_approx(x.y);
       }
       acc[t & 3] = f2_add(acc[t & 3], f2(p0, p1));
-      pk[t] = pack_bf16x2(p0, p1);
+      if constexpr (F16)
+        pk[t] = pack_f16x2(p0 * pmul, p1 * pmul);
+      else
+        pk[t] = pack_bf16x2(p0, p1);
     }
     tmem_st16(S + c4 * 16, pk);
   }
@@ -127,11 +178,12 @@ __device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, f
   return a.x + a.y;
 }
 
-template <int D, int STAGES, int EMU>
-__global__ void __launch_bounds__(kThreadsFwd, 1)
+template <int D, int STAGES, int EMU, bool F8>
+__global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
-  using Smem = FwdSmem<D, STAGES>;
+  using Smem = FwdSmem<D, STAGES, F8>;
+  constexpr int EB = F8 ? 1 : 2;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -152,10 +204,20 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       mbar_init(smem_u32(&sm.o_final[i]), 1);
       mbar_init(smem_u32(&sm.o_free[i]), 128);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.v16_full[i]), 2);  // one arrival per converter warp
+      mbar_init(smem_u32(&sm.v16_empty[i]), 1);
+    }
+    if constexpr (F8) {
+      // V tiles sit in the odd ring slots and are released by the two
+      // converter warps instead of an MMA commit
+      for (int s = 1; s < STAGES; s += 2) mbar_init(smem_u32(&sm.kv_empty[s]), 2);
+    }
     mbar_init(smem_u32(&sm.drain), 1);
     sm.abort = 0;
     fence_barrier_init();
   }
+  constexpr int kThreads = F8 ? kThreadsFwdF8 : kThreadsFwd;
   const int nlevels = (args.N + 255) / 256;
   const bool varlen = args.cu_seqlens != nullptr;
   if (warp == 9) {
@@ -170,7 +232,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   __syncthreads();
   int num_units = args.num_units;
   if (varlen)
-    num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 8, args.Hq, kThreadsFwd);
+    num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 8, args.Hq, kThreads);
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 8};
@@ -198,8 +260,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         const uint32_t qbar = smem_u32(&sm.q_full);
         mbar_expect_tx(qbar, 2 * Smem::kTileBytes);
         const int row0 = un.tok0 + un.qb2 * 2 * kBM;
-        load_tile<D>(smem_u32(sm.q[0]), &tm_q, qbar, un.h, row0);
-        load_tile<D>(smem_u32(sm.q[1]), &tm_q, qbar, un.h, row0 + kBM);
+        load_tile<D, EB>(smem_u32(sm.q[0]), &tm_q, qbar, un.h, row0);
+        load_tile<D, EB>(smem_u32(sm.q[1]), &tm_q, qbar, un.h, row0 + kBM);
         q_issued = it + 1;
         for (int j = 0; j < nblk && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
@@ -214,7 +276,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             } else {
               const uint32_t bar = smem_u32(&sm.kv_full[slot]);
               mbar_expect_tx(bar, Smem::kTileBytes);
-              load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
+              load_tile<D, EB>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
             }
             ++kv_prod;
           }
@@ -226,7 +288,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   } else if (warp == 9) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
-      uint32_t kv_cons = 0, it = 0, pc0 = 0, pc1 = 0;
+      uint32_t kv_cons = 0, it = 0, pc0 = 0, pc1 = 0, g = 0;
       bool ok = true;
       const uint32_t S0 = tmem + 0, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 384;
       auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
@@ -247,30 +309,34 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         uint32_t slotK = kv_cons % STAGES;
         if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 11))) break;
         ++kv_cons;
-        issue_qk<D>(S0, q0, smem_u32(sm.kv[slotK]));
+        issue_qk<D, F8>(S0, q0, smem_u32(sm.kv[slotK]));
         tc_commit(smem_u32(&sm.s_full[0]));
-        issue_qk<D>(S1, q1, smem_u32(sm.kv[slotK]));
+        issue_qk<D, F8>(S1, q1, smem_u32(sm.kv[slotK]));
         tc_commit(smem_u32(&sm.s_full[1]));
         tc_commit(smem_u32(&sm.kv_empty[slotK]));
         if (nblk == 1) tc_commit(smem_u32(&sm.q_empty));
-        for (int j = 0; j < nblk; ++j) {
+        for (int j = 0; j < nblk; ++j, ++g) {
           const bool has_next = j + 1 < nblk;
           const uint32_t slotV = kv_cons % STAGES;
-          if (!(ok = wait(&sm.kv_full[slotV], (kv_cons / STAGES) & 1, 12))) break;
+          if constexpr (F8) {
+            if (!(ok = wait(&sm.v16_full[g & 1], (g >> 1) & 1, 18))) break;
+          } else {
+            if (!(ok = wait(&sm.kv_full[slotV], (kv_cons / STAGES) & 1, 12))) break;
+          }
           ++kv_cons;
           if (has_next) {
             slotK = kv_cons % STAGES;
             if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 13))) break;
             ++kv_cons;
           }
-          const uint32_t vaddr = smem_u32(sm.kv[slotV]);
+          const uint32_t vaddr = F8 ? smem_u32(sm.v16[g & 1]) : smem_u32(sm.kv[slotV]);
           // ---- tile 0
           if (!(ok = wait(&sm.p_full[0], pc0 & 1, 14))) break;
           ++pc0;
           if (j == 0 && !(ok = wait(&sm.o_free[0], (it & 1) ^ 1, 15))) break;
-          issue_pv<D>(O0, S0, vaddr, j > 0);
+          issue_pv<D, F8>(O0, S0, vaddr, j > 0);
           if (has_next) {
-            issue_qk<D>(S0, q0, smem_u32(sm.kv[slotK]));
+            issue_qk<D, F8>(S0, q0, smem_u32(sm.kv[slotK]));
             tc_commit(smem_u32(&sm.s_full[0]));
           } else {
             tc_commit(smem_u32(&sm.o_final[0]));
@@ -279,10 +345,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           if (!(ok = wait(&sm.p_full[1], pc1 & 1, 16))) break;
           ++pc1;
           if (j == 0 && !(ok = wait(&sm.o_free[1], (it & 1) ^ 1, 17))) break;
-          issue_pv<D>(O1, S1, vaddr, j > 0);
-          tc_commit(smem_u32(&sm.kv_empty[slotV]));
+          issue_pv<D, F8>(O1, S1, vaddr, j > 0);
+          tc_commit(F8 ? smem_u32(&sm.v16_empty[g & 1]) : smem_u32(&sm.kv_empty[slotV]));
           if (has_next) {
-            issue_qk<D>(S1, q1, smem_u32(sm.kv[slotK]));
+            issue_qk<D, F8>(S1, q1, smem_u32(sm.kv[slotK]));
             tc_commit(smem_u32(&sm.s_full[1]));
             tc_commit(smem_u32(&sm.kv_empty[slotK]));
             if (j + 2 == nblk) tc_commit(smem_u32(&sm.q_empty));
@@ -296,6 +362,42 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       tc_commit(smem_u32(&sm.drain));
       mbar_wait(smem_u32(&sm.drain), 0, nullptr, args.timeout_ns);
     }
+  } else if (warp >= 10) {
+    // ======================= fp8: V widening warps =======================
+    if constexpr (F8) {
+      const int t = tid - 10 * 32;
+      uint32_t g = 0, it = 0;
+      bool ok = true;
+      for (int rnd = 0; ok; ++rnd, ++it) {
+        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (u >= num_units) break;
+        const Unit un = decode_unit(sched, u);
+        const int nblk = num_kv_blocks(un, args.causal);
+        for (int j = 0; j < nblk; ++j, ++g) {
+          const uint32_t idx = 2 * g + 1;  // ring index of V_j (K and V alternate)
+          const uint32_t slot = idx % STAGES;
+          ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.kv_full[slot]), (idx / STAGES) & 1, abort,
+                                                 args.timeout_ns));
+          if (ok)
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.v16_empty[g & 1]), ((g >> 1) & 1) ^ 1, abort,
+                                                   args.timeout_ns));
+          if (!ok) {
+            if (lane == 0) report_error(args.status, kStatusTimeout, 25);
+            break;
+          }
+          // warp w widens keys 64*(w-10) .. +63
+          widen_v_tile<D>(sm.kv[slot] + (warp - 10) * 64 * 128, sm.v16[g & 1] + (warp - 10) * 64 * 128, lane, 32, 64);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&sm.v16_full[g & 1]));
+            mbar_arrive(smem_u32(&sm.kv_empty[slot]));
+          }
+        }
+      }
+      if (!ok) sm.abort = 1;
+      (void)t;
+    }
   } else {
     // ======================= softmax warpgroups =======================
     const int tile = warp >> 2;               // 0 or 1
@@ -305,17 +407,35 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const uint32_t S = tmem + tile * 128 + lane_bits;
     const uint32_t O = tmem + 256 + tile * 128 + lane_bits;
     const float cl = args.scale_log2;
+    constexpr float tau = kTau;
     uint32_t sc = 0, it = 0;
     bool ok = true;
     for (int rnd = 0; ok; ++rnd, ++it) {
-        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
-        if (u >= num_units) break;
+      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
       const int nblk = num_kv_blocks(un, args.causal);
       const int row = un.qb2 * 2 * kBM + tile * kBM + r_in_tile;  // row within the sequence
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;  // last visible key
+      // scores are kept in base-2 units t = s * cj; cj = scale*log2(e) for
+      // bf16, times the query and key block scales for fp8
+      float sq = 1.f, sv_max = 1.f;
+      size_t kvs = 0;
+      if constexpr (F8) {
+        const int qt = un.qb2 * 2 + tile;
+        if (qt < args.nblk_s) sq = args.q_scale[(static_cast<size_t>(un.seq) * args.Hq + un.h) * args.nblk_s + qt];
+        kvs = (static_cast<size_t>(un.seq) * args.Hkv + un.h / group) * args.nblk_s;
+        sv_max = 0.f;
+        for (int jj = 0; jj < nblk; ++jj) sv_max = fmaxf(sv_max, args.v_scale[kvs + jj]);
+        sv_max = fmaxf(sv_max, 1e-30f);
+      }
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nblk; ++j) {
+        float cj = cl, pmul = 1.f;
+        if constexpr (F8) {
+          cj = cl * sq * args.k_scale[kvs + j];
+          pmul = args.v_scale[kvs + j] / sv_max;
+        }
         // every lane waits; the outcome is made warp-uniform so that the
         // warp-collective tcgen05 loads below run converged
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[tile]), sc & 1, abort, args.timeout_ns));
@@ -346,10 +466,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           for (int c = 3; c + 1 < 32; c += 2) a = fmax3(a, s[q4 * 32 + c], s[q4 * 32 + c + 1]);
           mx[q4] = fmaxf(a, s[q4 * 32 + 31]);
         }
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        const bool need = (mt - m) * cl > kTau;
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * cj;
+        const bool need = mt - m > tau;
         const float m_new = need ? mt : m;
-        const float alpha = need ? ex2_approx((m - m_new) * cl) : 1.f;
+        const float alpha = need ? ex2_approx(m - m_new) : 1.f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O rows whose maximum moved are rescaled in TMEM; the PV MMA of
           // the previous block has completed (it precedes this S in issue
@@ -363,9 +483,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
             tmem_st32(O + c, orr);
           }
         }
-        // P = 2^(s*c - m*c), written as bf16 over the first 64 columns of S
-        const float lsum = masked_blk ? softmax_exp_store<0>(s, S, cl, m_new * cl)
-                                      : softmax_exp_store<EMU>(s, S, cl, m_new * cl);
+        // P = 2^(s*cj - m), written over the first TMEM columns of S
+        const float lsum = masked_blk ? softmax_exp_store<0, F8>(s, S, cj, m_new, pmul)
+                                      : softmax_exp_store<EMU, F8>(s, S, cj, m_new, pmul);
         l = l * alpha + lsum;
         m = m_new;
         tmem_st_wait();
@@ -381,7 +501,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       }
       tc_fence_after();
       const bool valid = row < un.n;
-      const float inv_l = 1.f / l;
+      // fp8: P entered the PV MMA scaled by sv_j / sv_max
+      const float inv_l = (F8 ? sv_max : 1.f) / l;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
                             (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D;
 #pragma unroll 1
@@ -403,7 +524,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       if (valid) {
         const size_t li = varlen ? (static_cast<size_t>(un.h) * args.lse_head_stride + un.tok0 + row)
                                  : (static_cast<size_t>(un.seq * args.Hq + un.h) * args.lse_head_stride + row);
-        args.lse[li] = m * args.scale + logf(l);
+        args.lse[li] = m * 0.6931471805599453f + logf(l);
       }
     }
     if (!ok) sm.abort = 1;
