@@ -98,9 +98,10 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
 
 /*
  * Bytes of device workspace fa_bwd / fa_bwd_varlen need: two fp32 vectors per
- * (query head, token), the row's LSE in base 2 and D = dot(dO, O), with 128
- * padding rows per head. tokens = B*N (padded) or total_T (varlen); nseq and
- * d do not change the size (kept for a stable signature). 0 for empty inputs.
+ * (query head, token), the row's LSE in base 2 and D = dot(dO, O); each
+ * sequence's rows start 16-byte aligned, plus 128 padding rows per head.
+ * tokens = B*N (padded) or total_T (varlen); nseq = B or the number of packed
+ * sequences; d does not change the size. 0 for empty inputs.
  */
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
 
@@ -145,8 +146,8 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
  *   Arguments and results as fa_bwd, minus the workspace: the scratch lives in
  *   an 8 MiB array inside the library, on every device that loads it, for the
  *   life of the process. The problem must fit it:
- *   fa_bwd_workspace_size(B*N, B, Hq, d) <= 8 MiB, i.e. Hq * (B*N + 128) up
- *   to about 1.04 million; larger problems return FA_ERR_WORKSPACE and launch
+ *   fa_bwd_workspace_size(B*N, B, Hq, d) <= 8 MiB, i.e. Hq * (B*N + 4*B + 131)
+ *   up to about 1.04 million; larger problems return FA_ERR_WORKSPACE and launch
  *   nothing.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call

@@ -182,8 +182,12 @@ fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, f
   return FA_ERR_UNSUPPORTED;
 }
 
-size_t vec_bytes(int tokens, int Hq) {
-  const size_t b = static_cast<size_t>(Hq) * (static_cast<size_t>(tokens) + fa::kVecSlack) * sizeof(float);
+// Floats per head of each backward workspace vector (see fa::ws_offset).
+size_t vec_stride(int tokens, int nseq) {
+  return ((static_cast<size_t>(tokens) + 3) & ~size_t(3)) + 4 * static_cast<size_t>(nseq) + fa::kVecSlack;
+}
+size_t vec_bytes(int tokens, int nseq, int Hq) {
+  const size_t b = static_cast<size_t>(Hq) * vec_stride(tokens, nseq) * sizeof(float);
   return (b + 255) & ~size_t(255);
 }
 
@@ -249,7 +253,7 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
       !aligned(dv, 16))
     return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  const size_t vb = vec_bytes(total_T, Hq);
+  const size_t vb = vec_bytes(total_T, nseq, Hq);
   if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < 2 * vb) return FA_ERR_WORKSPACE;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
@@ -272,7 +276,8 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   a.scale = scale;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   a.lse_head_stride = cu ? total_T : N;
-  a.ws_stride = total_T + fa::kVecSlack;
+  if (vec_stride(total_T, nseq) > static_cast<size_t>(INT32_MAX)) return FA_ERR_UNSUPPORTED;
+  a.ws_stride = static_cast<int>(vec_stride(total_T, nseq));
   const long long nt = (N + 127) / 128;
   long long udq, ukv;
   if (cu == nullptr) {
@@ -377,10 +382,9 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
 }
 
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
-  (void)nseq;
   (void)d;
-  if (tokens <= 0 || Hq <= 0) return 0;
-  return 2 * vec_bytes(tokens, Hq);
+  if (tokens <= 0 || Hq <= 0 || nseq < 0) return 0;
+  return 2 * vec_bytes(tokens, nseq, Hq);
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,

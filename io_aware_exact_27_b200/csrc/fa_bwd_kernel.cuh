@@ -37,8 +37,8 @@ struct BwdArgs {
   void* dq;
   void* dk;
   void* dv;
-  float* lse2;          // workspace [Hq][total_T + 128]: LSE * log2(e), +inf past the end
-  float* dvec;          // workspace [Hq][total_T + 128]: D, 0 past the end
+  float* lse2;          // workspace [Hq][ws_stride]: LSE * log2(e), +inf where no token
+  float* dvec;          // workspace [Hq][ws_stride]: D, 0 where no token
   const int* cu_seqlens;
   int nseq;             // padded: B
   int N;                // padded: N; varlen: max_seqlen
@@ -48,16 +48,24 @@ struct BwdArgs {
   float scale;
   float scale_log2;
   int lse_head_stride;  // forward LSE: padded N, varlen total_T
-  int ws_stride;        // total_T + 128
+  int ws_stride;        // round_up4(total_T) + 4 * nseq + 128 (see ws_offset)
   int num_units;
   uint64_t timeout_ns;
   int* status;
 };
 
 // ------------------------------------------------------------------ pre
-// One warp per (head, token) row: D = dot(dO, O) in fp32 and LSE in base 2.
-// The 128 slack entries per head hold +inf (LSE) and 0 (D) so that tile
-// loads past a sequence end read harmless values.
+// Workspace layout: per query head, sequence s's rows start at
+//   ws_offset(s) = round_up(first token of s, 4) + 4 * s,
+// a 16-byte aligned float offset, so that the 128-row vectors of a query
+// tile can be fetched with one bulk copy; gaps and the 128 trailing entries
+// per head hold +inf (LSE) and 0 (D), harmless when a tile runs past the end
+// of its sequence.
+__device__ __forceinline__ int ws_offset(int tok0, int seq) { return ((tok0 + 3) & ~3) + 4 * seq; }
+
+// One warp per workspace entry (head, i): finds the sequence holding entry i
+// (binary search over the sequence starts), then D = dot(dO, O) in fp32 and
+// the base-2 LSE of that token, or the filler values.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
   const int lane = threadIdx.x & 31;
@@ -67,14 +75,25 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
   constexpr int PER = D / 32;  // elements per lane
   for (long long r = w0; r < rows; r += nw) {
     const int h = static_cast<int>(r / a.ws_stride);
-    const int tok = static_cast<int>(r - static_cast<long long>(h) * a.ws_stride);
-    if (tok >= a.total_T) {
+    const int i = static_cast<int>(r - static_cast<long long>(h) * a.ws_stride);
+    // last sequence whose workspace block starts at or before i
+    int lo = 0, hi = a.nseq - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + mid) : mid * a.N;
+      if (ws_offset(t0, mid) <= i) lo = mid; else hi = mid - 1;
+    }
+    const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + lo) : lo * a.N;
+    const int n = a.cu_seqlens ? __ldg(a.cu_seqlens + lo + 1) - t0 : a.N;
+    const int row = i - ws_offset(t0, lo);
+    if (row < 0 || row >= n) {
       if (lane == 0) {
         a.lse2[r] = INFINITY;
         a.dvec[r] = 0.f;
       }
       continue;
     }
+    const int tok = t0 + row;
     const size_t base = (static_cast<size_t>(tok) * a.Hq + h) * D + lane * PER;
     const __nv_bfloat16* op = reinterpret_cast<const __nv_bfloat16*>(a.o) + base;
     const __nv_bfloat16* gp = reinterpret_cast<const __nv_bfloat16*>(a.dout) + base;
@@ -101,13 +120,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
-      size_t li;
-      if (a.cu_seqlens != nullptr) {
-        li = static_cast<size_t>(h) * a.lse_head_stride + tok;
-      } else {
-        const int b = tok / a.N;
-        li = (static_cast<size_t>(b) * a.Hq + h) * a.lse_head_stride + (tok - b * a.N);
-      }
+      const size_t li = a.cu_seqlens ? static_cast<size_t>(h) * a.lse_head_stride + tok
+                                     : (static_cast<size_t>(lo) * a.Hq + h) * a.lse_head_stride + row;
       a.lse2[r] = a.lse[li] * kLog2e;
       a.dvec[r] = acc;
     }
@@ -318,7 +332,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
       const int row = un.qb2 * kBM + r_in_tile;
       const bool valid = row < un.n;
-      const size_t wi = static_cast<size_t>(un.h) * args.ws_stride + un.tok0 + row;
+      const size_t wi = static_cast<size_t>(un.h) * args.ws_stride + ws_offset(un.tok0, un.seq) + row;
       const float lse2 = valid ? args.lse2[wi] : INFINITY;
       const float dval = valid ? args.dvec[wi] : 0.f;
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;
@@ -420,7 +434,7 @@ struct DkvSmem {
   alignas(1024) uint8_t k[kTileBytes];
   alignas(1024) uint8_t v[kTileBytes];
   alignas(1024) uint8_t qo[STAGES][kTileBytes];  // Q_i, dO_i alternating
-  float vec[STAGES / 2][2][128];                 // per step: LSE2, D of the 128 query columns
+  alignas(16) float vec[STAGES / 2][2][128];     // per step: LSE2, D of the 128 query columns
   uint64_t kv_full, kv_empty;
   uint64_t qo_full[STAGES], qo_empty[STAGES];
   uint64_t s_full, dp_full, p_ready, ds_ready, acc_final, acc_free;
@@ -526,20 +540,18 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             if (lane == 0) report_error(args.status, kStatusTimeout, 61);
             break;
           }
-          if (w == 0) {
-            // the query tile's LSE2 and D, 4 each per lane
-            float* vec = sm.vec[(qo_prod / 2) % (STAGES / 2)][0];
-            const size_t wbase = static_cast<size_t>(hq) * args.ws_stride + un.tok0 + qi * kBM;
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              vec[lane + 32 * t] = args.lse2[wbase + lane + 32 * t];
-              vec[128 + lane + 32 * t] = args.dvec[wbase + lane + 32 * t];
-            }
-            __syncwarp();
-          }
           if (lane == 0) {
             const uint32_t bar = smem_u32(&sm.qo_full[slot]);
-            mbar_expect_tx(bar, Smem::kTileBytes);
+            if (w == 0) {
+              // the query tile's LSE2 and D ride on the Q tile's barrier
+              float* vec = sm.vec[(qo_prod / 2) % (STAGES / 2)][0];
+              const size_t wbase = static_cast<size_t>(hq) * args.ws_stride + ws_offset(un.tok0, un.seq) + qi * kBM;
+              mbar_expect_tx(bar, Smem::kTileBytes + 1024);
+              bulk_load(smem_u32(vec), args.lse2 + wbase, 512, bar);
+              bulk_load(smem_u32(vec + 128), args.dvec + wbase, 512, bar);
+            } else {
+              mbar_expect_tx(bar, Smem::kTileBytes);
+            }
             load_tile<D>(smem_u32(sm.qo[slot]), w == 0 ? &tm_q : &tm_do, bar, hq, un.tok0 + qi * kBM);
           }
           ++qo_prod;
@@ -577,6 +589,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (!(ok = wait(&sm.qo_full[slotO], ((qo_cons + 1) / STAGES) & 1, 72))) break;
         issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[slotO]));
         tc_commit(smem_u32(&sm.dp_full));
+        if (nsteps == 1) tc_commit(smem_u32(&sm.kv_empty));  // last reads of K and V issued
         qo_cons += 2;
         for (int st = 0; st < nsteps; ++st) {
           const bool has_next = st + 1 < nsteps;
@@ -585,6 +598,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           ++pc;
           if (st == 0 && !(ok = wait(&sm.acc_free, (it & 1) ^ 1, 74))) break;
           issue_ts_split<D>(tDV, tS, smem_u32(sm.qo[slotO]), st > 0);
+          tc_commit(smem_u32(&sm.qo_empty[slotO]));  // dO_st: last use
           uint32_t nQ = 0, nO = 0;
           if (has_next) {
             nQ = qo_cons % STAGES;
@@ -597,12 +611,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           if (!(ok = wait(&sm.ds_ready, dsc & 1, 76))) break;
           ++dsc;
           issue_ts_split<D>(tDK, tDP, smem_u32(sm.qo[slotQ]), st > 0);
-          tc_commit(smem_u32(&sm.qo_empty[slotQ]));
-          tc_commit(smem_u32(&sm.qo_empty[slotO]));
+          tc_commit(smem_u32(&sm.qo_empty[slotQ]));  // Q_st: last use
           if (has_next) {
             if (!(ok = wait(&sm.qo_full[nO], ((qo_cons + 1) / STAGES) & 1, 77))) break;
             issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[nO]));
             tc_commit(smem_u32(&sm.dp_full));
+            // K and V are last read by this unit's final S^T and dP^T: release
+            // them now so the next unit's tiles load under the last steps
+            if (st + 2 == nsteps) tc_commit(smem_u32(&sm.kv_empty));
             qo_cons += 2;
             slotQ = nQ;
             slotO = nO;
@@ -610,7 +626,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         }
         if (!ok) break;
         tc_commit(smem_u32(&sm.acc_final));
-        tc_commit(smem_u32(&sm.kv_empty));
       }
       if (!ok) sm.abort = 1;
       tc_commit(smem_u32(&sm.drain));

@@ -49,9 +49,11 @@ def test_status_strings(lib):
 def test_workspace_size_host_logic(lib):
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     ws = lib.fa_bwd_workspace_size(4 * 2048, 4, 16, 128)
-    # two fp32 vectors per query row and head (LSE in base 2 and dot(dO, O)),
-    # plus 128 rows of padding per head, each vector 256-byte aligned
-    assert ws == 2 * ((16 * (4 * 2048 + 128) * 4 + 255) // 256 * 256)
+    # two fp32 vectors per (query head, token) (LSE in base 2 and dot(dO, O));
+    # per head: tokens rounded up to 4, 4 floats of alignment room per
+    # sequence and 128 trailing entries; each vector 256-byte aligned
+    per_head = (4 * 2048 + 3) // 4 * 4 + 4 * 4 + 128
+    assert ws == 2 * ((16 * per_head * 4 + 255) // 256 * 256)
     assert ws % 256 == 0
     assert lib.fa_bwd_workspace_size(0, 1, 16, 128) == 0
 
