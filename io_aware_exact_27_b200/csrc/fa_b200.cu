@@ -22,7 +22,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 std::atomic<int> g_inject{0};
-std::atomic<int> g_exp_emu{2};  // pairs of every 8 whose exp2 runs on the FMA pipe
+std::atomic<int> g_exp_emu{0};  // pairs of every 8 whose exp2 runs on the FMA pipe
 std::atomic<int> g_last_word{0};
 
 constexpr int kMaxDevices = 64;

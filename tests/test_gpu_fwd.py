@@ -230,8 +230,8 @@ def test_exp_emulation_variants(fa, emu, causal):
     try:
         (q, k, v), o, lse = _run_padded(fa, 2, 1024, 4, 2, 128, causal, seed=17)
     finally:
-        fa.fa_set_exp_emulation(2)
+        fa.fa_set_exp_emulation(0)
     O, L = oracle.attn_fwd(q, k, v, causal, 1 / math.sqrt(128))
     _check_o_lse(o, lse, O, L, f"emu={emu}")
     with pytest.raises(fa.FAError):
-        fa.fa_set_exp_emulation(5)
+        fa.fa_set_exp_emulation(1)
