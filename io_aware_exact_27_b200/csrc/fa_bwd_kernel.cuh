@@ -153,10 +153,12 @@ __device__ __forceinline__ uint32_t split_a_col(int kk) { return kk < 4 ? 8 * kk
 template <int DD>
 __device__ __forceinline__ void issue_ts_split(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, DD, false, true);
+  const uint64_t bd = smem_desc(b_smem, 16384, 1024, kSwizzle128B);  // + (kk * 2048) >> 4 per step
+  const uint32_t acc0 = accumulate ? 1u : 0u;
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_f16_ts(d_tmem, a_tmem + split_a_col(kk), smem_desc(b_smem + kk * 2048, 16384, 1024, kSwizzle128B), idesc,
-               (accumulate || kk > 0) ? 1u : 0u);
+    mma_f16_ts(d_tmem, a_tmem + split_a_col(kk), bd + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+               kk > 0 ? 1u : acc0);
 }
 
 // D(128 x 128) = A(smem [128 x DD] K-major) * B(smem [128 x DD] K-major)^T

@@ -81,20 +81,24 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m, ui
   for (int b = 0; b < D * EB / 128; ++b) tma_load_3d(dst + b * 16384, m, bar, b * (128 / EB), head, row0);
 }
 
+// Descriptors are built once per call; each MMA adds a compile-time byte
+// offset (>> 4) to the 14-bit start-address field. Shared-memory addresses
+// stay below 228 KB, so (address + offset) >> 4 never leaves the field.
+
 // S = Q K^T over d: each MMA consumes 32 bytes of every row (16 bf16 or 32
 // e4m3 elements), advancing inside the 128-byte swizzle row.
 template <int D, bool F8 = false>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
   constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(kBM, kBN, false, false) : idesc_bf16_f32(kBM, kBN, false, false);
+  const uint64_t qd = smem_desc(q_smem, 16, 1024, kSwizzle128B);
+  const uint64_t kd = smem_desc(k_smem, 16, 1024, kSwizzle128B);
 #pragma unroll
   for (int kk = 0; kk < D * (F8 ? 1 : 2) / 32; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    const uint64_t a = smem_desc(q_smem + off, 16, 1024, kSwizzle128B);
-    const uint64_t b = smem_desc(k_smem + off, 16, 1024, kSwizzle128B);
+    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
     if constexpr (F8)
-      mma_f8_ss(s_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+      mma_f8_ss(s_tmem, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
     else
-      mma_f16_ss(s_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+      mma_f16_ss(s_tmem, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -104,10 +108,11 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
 template <int D, bool F16 = false>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = F16 ? idesc_f16_f32(kBM, D, false, true) : idesc_bf16_f32(kBM, D, false, true);
+  const uint64_t vd = smem_desc(v_smem, 16384, 1024, kSwizzle128B);
+  const uint32_t acc0 = accumulate ? 1u : 0u;
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_f16_ts(o_tmem, p_tmem + kk * 8, smem_desc(v_smem + kk * 2048, 16384, 1024, kSwizzle128B), idesc,
-               (accumulate || kk > 0) ? 1u : 0u);
+    mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc, kk > 0 ? 1u : acc0);
 }
 
 // fp8: widens `nkeys` rows (keys) of an e4m3 V tile to f16 (exactly) in the
@@ -141,38 +146,31 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
 }
 
-// Exponentials of one 128-column row slice: p = 2^(s*cj - m) in fp32 (the
-// row sum), stored over the first 64 TMEM columns of the S tile as the A
-// operand of the PV MMA: bf16 pairs, or (fp8 path) f16 pairs of p*pmul, the
-// V block scale folded in. Scale and sum run on packed fp32 pairs; EMU of
-// every 8 pairs take exp2 on the FMA pipe (exp2_poly_pair), the rest on MUFU.
+// Exponentials of 64 consecutive columns of one row: p = 2^(s*cj - m),
+// packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[32] for
+// the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs;
+// EMU of every 8 pairs take exp2 on the FMA pipe (exp2_poly_pair).
 template <int EMU, bool F16>
-__device__ __forceinline__ float softmax_exp_store(const float* s, uint32_t S, float cj, float m, float pmul) {
+__device__ __forceinline__ float exp_pack(const float* s, float cj, float m, float pmul, uint32_t* pk) {
   const uint64_t c2 = f2(cj, cj);
   const uint64_t nm2 = f2(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const int e = c4 * 32 + 2 * t;
-      const uint64_t x2 = f2_fma(f2(s[e], s[e + 1]), c2, nm2);
-      float p0, p1;
-      if ((t & 7) < EMU) {
-        exp2_poly_pair(x2, p0, p1);
-      } else {
-        const float2 x = f2_split(x2);
-        p0 = ex2_approx(x.x);
-        p1 = ex2_approx(x.y);
-      }
-      acc[t & 3] = f2_add(acc[t & 3], f2(p0, p1));
-      if constexpr (F16)
-        pk[t] = pack_f16x2(p0 * pmul, p1 * pmul);
-      else
-        pk[t] = pack_bf16x2(p0, p1);
+  for (int t = 0; t < 32; ++t) {
+    const uint64_t x2 = f2_fma(f2(s[2 * t], s[2 * t + 1]), c2, nm2);
+    float p0, p1;
+    if ((t & 7) < EMU) {
+      exp2_poly_pair(x2, p0, p1);
+    } else {
+      const float2 x = f2_split(x2);
+      p0 = ex2_approx(x.x);
+      p1 = ex2_approx(x.y);
     }
-    tmem_st16(S + c4 * 16, pk);
+    acc[t & 3] = f2_add(acc[t & 3], f2(p0, p1));
+    if constexpr (F16)
+      pk[t] = pack_f16x2(p0 * pmul, p1 * pmul);
+    else
+      pk[t] = pack_bf16x2(p0, p1);
   }
   const float2 a = f2_split(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])));
   return a.x + a.y;
@@ -445,28 +443,32 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         }
         ++sc;
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld128(S, sr);
-        float* s = reinterpret_cast<float*>(sr);
         const int kv0 = j * kBN;
-        // Warp-uniform: the exponential path below holds warp-collective
-        // TMEM stores, so every lane of a warp must take the same branch.
+        // Warp-uniform: the passes below hold warp-collective TMEM loads and
+        // stores, so every lane of a warp must take the same branch.
         const bool masked_blk = __any_sync(0xffffffffu, kv0 + kBN - 1 > limit);
-        if (masked_blk) {
+        // pass 1: row maximum, 64 columns at a time (keeps register use low)
+        float mh[2];
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (kv0 + c > limit) s[c] = -INFINITY;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld64(S + 64 * h, sr);
+          float* sv = reinterpret_cast<float*>(sr);
+          if (masked_blk) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (kv0 + 64 * h + c > limit) sv[c] = -INFINITY;
+          }
+          float a = fmax3(sv[0], sv[1], sv[2]);
+          float b = fmax3(sv[32], sv[33], sv[34]);
+#pragma unroll
+          for (int c = 3; c < 31; c += 2) {
+            a = fmax3(a, sv[c], sv[c + 1]);
+            b = fmax3(b, sv[32 + c], sv[32 + c + 1]);
+          }
+          mh[h] = fmax3(fmaxf(a, sv[31]), b, sv[63]);
         }
-        // row maximum: four independent chains of three-input max
-        float mx[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float a = fmax3(s[q4 * 32 + 0], s[q4 * 32 + 1], s[q4 * 32 + 2]);
-#pragma unroll
-          for (int c = 3; c + 1 < 32; c += 2) a = fmax3(a, s[q4 * 32 + c], s[q4 * 32 + c + 1]);
-          mx[q4] = fmaxf(a, s[q4 * 32 + 31]);
-        }
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * cj;
+        const float mt = fmaxf(mh[0], mh[1]) * cj;
         const bool need = mt - m > tau;
         const float m_new = need ? mt : m;
         const float alpha = need ? ex2_approx(m - m_new) : 1.f;
@@ -483,9 +485,25 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
             tmem_st32(O + c, orr);
           }
         }
-        // P = 2^(s*cj - m), written over the first TMEM columns of S
-        const float lsum = masked_blk ? softmax_exp_store<0, F8>(s, S, cj, m_new, pmul)
-                                      : softmax_exp_store<EMU, F8>(s, S, cj, m_new, pmul);
+        // pass 2: P = 2^(s*cj - m), 64 columns at a time. The first half's P
+        // lands on columns [0,32) (already read), the second half's on
+        // [32,64) (read in the first half), so no S value is overwritten early.
+        float lsum = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[64];
+          tmem_ld64(S + 64 * h, sr);
+          float* sv = reinterpret_cast<float*>(sr);
+          if (masked_blk) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (kv0 + 64 * h + c > limit) sv[c] = -INFINITY;
+          }
+          uint32_t pk[32];
+          lsum += masked_blk ? exp_pack<0, F8>(sv, cj, m_new, pmul, pk) : exp_pack<EMU, F8>(sv, cj, m_new, pmul, pk);
+          tmem_st16(S + 32 * h, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+          tmem_st16(S + 32 * h + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+        }
         l = l * alpha + lsum;
         m = m_new;
         tmem_st_wait();
