@@ -202,8 +202,9 @@ void fa_debug_set_inject(int mode);
  * MUFU): of every 8 pairs of score
  * elements, how many take their exponential on the FMA pipe (a cubic
  * polynomial after exact range reduction, relative error < 1e-4) instead of
- * the MUFU unit. Accepted: 0, 2, 3 (default 0, fastest when measured); other values return FA_ERR_UNSUPPORTED. Blocks that contain
- * masked keys always use MUFU. Affects launches made after the call.
+ * the MUFU unit. Accepted: 0, 2, 3 (default 0, the fastest measured); other
+ * values return FA_ERR_UNSUPPORTED. Blocks that contain masked keys always use
+ * MUFU. Affects launches made after the call.
  */
 fa_status_t fa_set_exp_emulation(int pairs_of_8);
 

@@ -32,7 +32,7 @@ struct DeviceState {
   int sms = 0;
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
-  bool fwd_attr[3][5] = {};
+  bool fwd_attr[3][6] = {};
   bool bwd_attr[2] = {false, false};
 };
 DeviceState g_dev[kMaxDevices];

@@ -144,10 +144,7 @@ struct DqSmem {
   int level_count[1024];
 };
 
-// A operand taken from TMEM where each elementwise column half stored its
-// bf16 pairs: 16-element K step kk of the first half at column 8*kk, of the
-// second half at column 64 + 8*(kk-4).
-__device__ __forceinline__ uint32_t split_a_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+// (split_a_col: the split TMEM A-operand layout, shared with the forward)
 
 // D(M=128, N=DD) (+)= A(TMEM, 128 x 128 split halves) * B(smem [128 x DD] MN-major)
 template <int DD>

@@ -9,11 +9,14 @@
 // attention matrix; Dao-AILab repository overview: online softmax with
 // rescaling, tiled attention, persistent tile schedulers).
 //
-// Design (one persistent CTA per SM, 320 threads):
-//   warps 0-3  softmax of query tile 0 (thread = row = TMEM lane)
-//   warps 4-7  softmax of query tile 1
-//   warp  8    TMA producer: Q tiles once per unit, K_j / V_j through a ring
-//   warp  9    tcgen05 issuer (one thread) and TMEM owner
+// Design (one persistent CTA per SM, 576 threads; 640 for fp8):
+//   warps 0-7   softmax of query tile 0: warp w takes TMEM lanes (rows)
+//               32*(w%4).. and key columns 64*((w/4)%2)..; the two warps of
+//               a row quadrant exchange row maxima and sums through smem
+//   warps 8-15  softmax of query tile 1, likewise
+//   warp  16    TMA producer: Q tiles once per unit, K_j / V_j through a ring
+//   warp  17    tcgen05 issuer (one thread) and TMEM owner
+//   warps 18-19 fp8 only: widen e4m3 V tiles to f16
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 // P (bf16) is written over the first 64 columns of its S tile and fed to the
 // PV MMA straight from TMEM. The two query tiles ping-pong: while one tile's
@@ -26,9 +29,15 @@ namespace fa {
 
 constexpr int kBM = 128;      // query rows per tile
 constexpr int kBN = 128;      // keys per block
-constexpr int kThreadsFwd = 320;
-// fp8 adds two warps that widen each e4m3 V tile to f16 for the PV MMA
-constexpr int kThreadsFwdF8 = 384;
+// Warp roles: 16 softmax warps (two per TMEM lane quadrant per query tile,
+// each on one half of the 128 key columns), the TMA producer, the MMA
+// issuer; fp8 adds two warps that widen each e4m3 V tile to f16.
+constexpr int kSoftmaxWarps = 16;
+constexpr int kWarpProducer = 16;
+constexpr int kWarpMma = 17;
+constexpr int kWarpConv = 18;
+constexpr int kThreadsFwd = 18 * 32;
+constexpr int kThreadsFwdF8 = 20 * 32;
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, base-2 exponent units
 
 
@@ -67,6 +76,8 @@ struct FwdSmem {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
   uint64_t v16_full[2], v16_empty[2];
+  uint64_t pair_bar[2][4];        // per (tile, lane quadrant): the two column halves
+  float xch[2][2][2][128];        // [slot][tile][half][row] values exchanged by a pair
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -102,9 +113,15 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
   }
 }
 
-// O += P V: P (bf16 or f16 pairs) read from TMEM, V a [keys, D] tile (D
-// contiguous) in shared memory as the MN-major B operand: LBO = next 64
-// columns of D (next 16 KB box), SBO = next 8 keys. One MMA covers 16 keys.
+// A operand taken from TMEM where each column half of the softmax stored its
+// 16-bit pairs: 16-key step kk of the first half at column 8*kk, of the
+// second half at column 64 + 8*(kk-4).
+__device__ __forceinline__ uint32_t split_a_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+
+// O += P V: P (bf16 or f16 pairs) read from TMEM in the split layout above,
+// V a [keys, D] tile (D contiguous) in shared memory as the MN-major B
+// operand: LBO = next 64 columns of D (next 16 KB box), SBO = next 8 keys.
+// One MMA covers 16 keys.
 template <int D, bool F16 = false>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = F16 ? idesc_f16_f32(kBM, D, false, true) : idesc_bf16_f32(kBM, D, false, true);
@@ -112,7 +129,8 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   const uint32_t acc0 = accumulate ? 1u : 0u;
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc, kk > 0 ? 1u : acc0);
+    mma_f16_ts(o_tmem, p_tmem + split_a_col(kk), vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+               kk > 0 ? 1u : acc0);
 }
 
 // fp8: widens `nkeys` rows (keys) of an e4m3 V tile to f16 (exactly) in the
@@ -146,17 +164,17 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
 }
 
-// Exponentials of 64 consecutive columns of one row: p = 2^(s*cj - m),
-// packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[32] for
+// Exponentials of 2*NP consecutive columns of one row: p = 2^(s*cj - m),
+// packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[NP] for
 // the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs;
 // EMU of every 8 pairs take exp2 on the FMA pipe (exp2_poly_pair).
-template <int EMU, bool F16>
+template <int EMU, bool F16, int NP = 32>
 __device__ __forceinline__ float exp_pack(const float* s, float cj, float m, float pmul, uint32_t* pk) {
   const uint64_t c2 = f2(cj, cj);
   const uint64_t nm2 = f2(-m, -m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int t = 0; t < 32; ++t) {
+  for (int t = 0; t < NP; ++t) {
     const uint64_t x2 = f2_fma(f2(s[2 * t], s[2 * t + 1]), c2, nm2);
     float p0, p1;
     if ((t & 7) < EMU) {
@@ -198,9 +216,10 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.s_full[i]), 1);
-      mbar_init(smem_u32(&sm.p_full[i]), 128);
+      mbar_init(smem_u32(&sm.p_full[i]), 8);  // one arrival per softmax warp of the tile
       mbar_init(smem_u32(&sm.o_final[i]), 1);
-      mbar_init(smem_u32(&sm.o_free[i]), 128);
+      mbar_init(smem_u32(&sm.o_free[i]), 8);
+      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&sm.pair_bar[i][q]), 2);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.v16_full[i]), 2);  // one arrival per converter warp
@@ -218,11 +237,11 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
   constexpr int kThreads = F8 ? kThreadsFwdF8 : kThreadsFwd;
   const int nlevels = (args.N + 255) / 256;
   const bool varlen = args.cu_seqlens != nullptr;
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
   uint32_t prod_issued = 0;  // K/V loads issued by the producer thread
   uint32_t q_issued = 0;     // Q loads issued by the producer thread
 
-  if (warp == 8) {
+  if (warp == kWarpProducer) {
     // ======================= TMA producer =======================
     if (lane == 0) {
       uint32_t kv_prod = 0, it = 0;
@@ -283,7 +302,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       if (!ok) sm.abort = 1;
       prod_issued = kv_prod;
     }
-  } else if (warp == 9) {
+  } else if (warp == kWarpMma) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
       uint32_t kv_cons = 0, it = 0, pc0 = 0, pc1 = 0, g = 0;
@@ -360,10 +379,10 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       tc_commit(smem_u32(&sm.drain));
       mbar_wait(smem_u32(&sm.drain), 0, nullptr, args.timeout_ns);
     }
-  } else if (warp >= 10) {
+  } else if (warp >= kWarpConv) {
     // ======================= fp8: V widening warps =======================
     if constexpr (F8) {
-      const int t = tid - 10 * 32;
+      const int t = tid - kWarpConv * 32;
       uint32_t g = 0, it = 0;
       bool ok = true;
       for (int rnd = 0; ok; ++rnd, ++it) {
@@ -383,8 +402,9 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
             if (lane == 0) report_error(args.status, kStatusTimeout, 25);
             break;
           }
-          // warp w widens keys 64*(w-10) .. +63
-          widen_v_tile<D>(sm.kv[slot] + (warp - 10) * 64 * 128, sm.v16[g & 1] + (warp - 10) * 64 * 128, lane, 32, 64);
+          // converter warp c widens keys 64*c .. +63
+          widen_v_tile<D>(sm.kv[slot] + (warp - kWarpConv) * 64 * 128, sm.v16[g & 1] + (warp - kWarpConv) * 64 * 128, lane,
+                          32, 64);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -396,18 +416,36 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       if (!ok) sm.abort = 1;
       (void)t;
     }
-  } else {
-    // ======================= softmax warpgroups =======================
-    const int tile = warp >> 2;               // 0 or 1
-    const int quad = warp & 3;                // TMEM lane quadrant
-    const int r_in_tile = quad * 32 + lane;   // TMEM lane = row within the tile
+  } else if (warp < kSoftmaxWarps) {
+    // ======================= softmax warps =======================
+    // warp w: query tile w/8, TMEM lane quadrant w%4 (row = lane), key column
+    // half (w/4)%2 of every 128-column S block
+    const int tile = warp >> 3;
+    const int quad = warp & 3;
+    const int half = (warp >> 2) & 1;
+    const int r_in_tile = quad * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t S = tmem + tile * 128 + lane_bits;
-    const uint32_t O = tmem + 256 + tile * 128 + lane_bits;
+    const uint32_t S = tmem + tile * 128 + 64 * half + lane_bits;          // this half of S
+    constexpr int HC = D / 2;                                              // O columns per half
+    const uint32_t O = tmem + 256 + tile * 128 + HC * half + lane_bits;    // this half of O
+    const uint32_t pair = smem_u32(&sm.pair_bar[tile][quad]);
     const float cl = args.scale_log2;
     constexpr float tau = kTau;
-    uint32_t sc = 0, it = 0;
+    uint32_t sc = 0, xc = 0, it = 0;
     bool ok = true;
+    // Hands v to the partner warp (same rows, other column half) and returns
+    // its value; two smem slots alternate so a fast warp never overwrites a
+    // value its partner has not read yet. Bounded wait; false on give-up.
+    auto exchange = [&](float v, float& other) -> bool {
+      const int slot = xc & 1;
+      sm.xch[slot][tile][half][r_in_tile] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pair);
+      const bool w = __all_sync(0xffffffffu, mbar_wait(pair, xc & 1, abort, args.timeout_ns));
+      ++xc;
+      other = sm.xch[slot][tile][half ^ 1][r_in_tile];
+      return w;
+    };
     for (int rnd = 0; ok; ++rnd, ++it) {
       const int u = unit_of(rnd, blockIdx.x, gridDim.x);
       if (u >= num_units) break;
@@ -427,7 +465,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         for (int jj = 0; jj < nblk; ++jj) sv_max = fmaxf(sv_max, args.v_scale[kvs + jj]);
         sv_max = fmaxf(sv_max, 1e-30f);
       }
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
       for (int j = 0; j < nblk; ++j) {
         float cj = cl, pmul = 1.f;
         if constexpr (F8) {
@@ -443,21 +481,19 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         }
         ++sc;
         tc_fence_after();
-        const int kv0 = j * kBN;
-        // Warp-uniform: the passes below hold warp-collective TMEM loads and
-        // stores, so every lane of a warp must take the same branch.
-        const bool masked_blk = __any_sync(0xffffffffu, kv0 + kBN - 1 > limit);
-        // pass 1: row maximum, 64 columns at a time (keeps register use low)
-        float mh[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        const int kv0 = j * kBN + 64 * half;  // first key of this half
+        // warp-uniform: every lane of a warp takes the same masked/unmasked path
+        const bool masked_blk = __any_sync(0xffffffffu, kv0 + 63 > limit);
+        // pass 1: this half's row maximum, exchanged with the partner half
+        float pm;
+        {
           uint32_t sr[64];
-          tmem_ld64(S + 64 * h, sr);
+          tmem_ld64(S, sr);
           float* sv = reinterpret_cast<float*>(sr);
           if (masked_blk) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
-              if (kv0 + 64 * h + c > limit) sv[c] = -INFINITY;
+              if (kv0 + c > limit) sv[c] = -INFINITY;
           }
           float a = fmax3(sv[0], sv[1], sv[2]);
           float b = fmax3(sv[32], sv[33], sv[34]);
@@ -466,18 +502,23 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
             a = fmax3(a, sv[c], sv[c + 1]);
             b = fmax3(b, sv[32 + c], sv[32 + c + 1]);
           }
-          mh[h] = fmax3(fmaxf(a, sv[31]), b, sv[63]);
+          pm = fmax3(fmaxf(a, sv[31]), b, sv[63]);
         }
-        const float mt = fmaxf(mh[0], mh[1]) * cj;
+        float po;
+        if (!exchange(pm, po)) {
+          ok = false;
+          if (lane == 0) report_error(args.status, kStatusTimeout, 24);
+          break;
+        }
+        const float mt = fmaxf(pm, po) * cj;  // identical in both halves
         const bool need = mt - m > tau;
         const float m_new = need ? mt : m;
         const float alpha = need ? ex2_approx(m - m_new) : 1.f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O rows whose maximum moved are rescaled in TMEM; the PV MMA of
-          // the previous block has completed (it precedes this S in issue
-          // order), so O is quiescent here.
+          // this half's O columns are rescaled in TMEM; the PV MMA of the
+          // previous block has completed (it precedes this S in issue order)
 #pragma unroll 1
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < HC; c += 32) {
             uint32_t orr[32];
             tmem_ld32(O + c, orr);
 #pragma unroll
@@ -485,46 +526,53 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
             tmem_st32(O + c, orr);
           }
         }
-        // pass 2: P = 2^(s*cj - m), 64 columns at a time. The first half's P
-        // lands on columns [0,32) (already read), the second half's on
-        // [32,64) (read in the first half), so no S value is overwritten early.
+        // pass 2: P = 2^(s*cj - m) in two 32-column chunks; chunk c's P pairs
+        // go to columns [16c, 16c+16) of this half, already read
         float lsum = 0.f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[64];
-          tmem_ld64(S + 64 * h, sr);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(S + 32 * c, sr);
           float* sv = reinterpret_cast<float*>(sr);
           if (masked_blk) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (kv0 + 64 * h + c > limit) sv[c] = -INFINITY;
+            for (int e = 0; e < 32; ++e)
+              if (kv0 + 32 * c + e > limit) sv[e] = -INFINITY;
           }
-          uint32_t pk[32];
-          lsum += masked_blk ? exp_pack<0, F8>(sv, cj, m_new, pmul, pk) : exp_pack<EMU, F8>(sv, cj, m_new, pmul, pk);
-          tmem_st16(S + 32 * h, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-          tmem_st16(S + 32 * h + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+          uint32_t pk[16];
+          lsum += masked_blk ? exp_pack<0, F8, 16>(sv, cj, m_new, pmul, pk)
+                             : exp_pack<EMU, F8, 16>(sv, cj, m_new, pmul, pk);
+          tmem_st16(S + 16 * c, pk);
         }
         l = l * alpha + lsum;
         m = m_new;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sm.p_full[tile]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[tile]));
       }
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16, LSE
+      // ---- epilogue: O / l -> bf16 (this half's columns), LSE
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[tile]), it & 1, abort, args.timeout_ns));
       if (!ok) {
         if (lane == 0) report_error(args.status, kStatusTimeout, 22 + tile);
         break;
       }
       tc_fence_after();
+      float lo;
+      if (!exchange(l, lo)) {
+        ok = false;
+        if (lane == 0) report_error(args.status, kStatusTimeout, 26);
+        break;
+      }
+      const float lt = l + lo;
       const bool valid = row < un.n;
       // fp8: P entered the PV MMA scaled by sv_j / sv_max
-      const float inv_l = (F8 ? sv_max : 1.f) / l;
+      const float inv_l = (F8 ? sv_max : 1.f) / lt;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
-                            (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D;
+                            (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D + HC * half;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < HC; c += 32) {
         uint32_t orr[32];
         tmem_ld32(O + c, orr);
         uint32_t pk[16];
@@ -538,11 +586,12 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.o_free[tile]));
-      if (valid) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.o_free[tile]));
+      if (valid && half == 0) {
         const size_t li = varlen ? (static_cast<size_t>(un.h) * args.lse_head_stride + un.tok0 + row)
                                  : (static_cast<size_t>(un.seq * args.Hq + un.h) * args.lse_head_stride + row);
-        args.lse[li] = m * 0.6931471805599453f + logf(l);
+        args.lse[li] = m * 0.6931471805599453f + logf(lt);
       }
     }
     if (!ok) sm.abort = 1;
@@ -551,7 +600,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
   // ---- teardown: every role is out of its loop; release TMEM
   tc_fence_before();
   __syncthreads();
-  if (sm.abort && warp == 8 && lane == 0) {
+  if (sm.abort && warp == kWarpProducer && lane == 0) {
     // after an abort, let the K/V loads already issued land before the CTA
     // exits (the newest load of each ring slot is the one still in flight)
     for (uint32_t i = (prod_issued > STAGES ? prod_issued - STAGES : 0); i < prod_issued; ++i) {
@@ -561,7 +610,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     if (q_issued > 0) mbar_wait(smem_u32(&sm.q_full), (q_issued - 1) & 1, nullptr, args.timeout_ns);
   }
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -214,7 +214,7 @@ def test_bounded_wait_reports_timeout(fa):
     assert st == fa.FA_ERR_TIMEOUT
     # the first wait to run out may be the MMA issuer's (K tile never loaded),
     # the producer's (ring slot never released) or a softmax warp's
-    assert (fa.fa_last_device_error_word() >> 8) & 0xff in (1, 2, 10, 11, 12, 13, 14, 20, 21)
+    assert (fa.fa_last_device_error_word() >> 8) & 0xff in (1, 2, 10, 11, 12, 13, 14, 20, 21, 24, 26)
     o, lse = fa.attention_fwd(q, k, v, causal=False)
     assert fa.fa_get_status() == fa.FA_OK
     O, L = oracle.attn_fwd(q.cpu(), k.cpu(), v.cpu(), False, 1 / math.sqrt(d))
