@@ -207,3 +207,42 @@ def dequantize_blockscaled(codes, scales, block: int = 128):
     blk = np.arange(N) // block
     per_row = s[:, :, blk]  # [B,H,N]
     return c * per_row.transpose(0, 2, 1)[..., None]
+
+
+def attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal: bool, scale: float):
+    """Attention of a few new query rows against a key/value cache (decode).
+
+    q [B,Nq,Hq,d]; k_cache, v_cache [B,Ncache,Hkv,d]; cache_seqlens [B]: batch
+    b holds L_b valid cache rows (keys 0 .. L_b-1). The queries are the newest
+    Nq positions of the sequence: query i sits at position L_b - Nq + i, so
+    with causal=True it sees keys 0 .. L_b - Nq + i (readings: the KV-cache API
+    of the Dao-AILab repository overview is named there without semantics;
+    bottom-right alignment is the decode convention where the newest query
+    sees the whole cache). A row that sees no key has O = 0, LSE = -inf.
+    Returns O [B,Nq,Hq,d], LSE [B,Hq,Nq] (float64).
+    """
+    q, k, v = _f64(q), _f64(k_cache), _f64(v_cache)
+    L = np.asarray(cache_seqlens, dtype=np.int64)
+    B, Nq, Hq, d = q.shape
+    Hkv = k.shape[2]
+    O = np.zeros((B, Nq, Hq, v.shape[3]))
+    LSE = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        Lb = int(L[b])
+        if Lb <= 0:
+            continue
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            S = scale * (q[b, :, h] @ k[b, :Lb, g].T)  # [Nq, Lb]
+            if causal:
+                pos = Lb - Nq + np.arange(Nq)
+                S = np.where(np.arange(Lb)[None, :] > pos[:, None], -np.inf, S)
+            for i in range(Nq):
+                row = S[i]
+                if not np.any(np.isfinite(row)):
+                    continue
+                m = row.max()
+                lse = m + np.log(np.exp(row - m).sum())
+                O[b, i, h] = np.exp(row - lse) @ v[b, :Lb, g]
+                LSE[b, h, i] = lse
+    return O, LSE

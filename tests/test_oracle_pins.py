@@ -286,3 +286,56 @@ def test_fp8_synth_roundtrip_error_bounded():
     rel = np.abs(x - xh) / np.maximum(np.abs(x), 1e-30)
     small = np.abs(x) < 2 ** -6 * d["q_scale"].numpy().max()
     assert np.all(rel[~small] <= 2 ** -4 + 1e-7)
+
+
+# --- decode against a KV cache (bottom-right causal alignment) -------------
+
+def test_kvcache_full_cache_equals_causal_self_attention():
+    """With Nq = L = Ncache every row of the cache is a query: the causal
+    decode result is ordinary causal attention."""
+    B, N, Hq, Hkv, d = 2, 9, 4, 2, 8
+    q, k, v = _rand((B, N, Hq, d), 60), _rand((B, N, Hkv, d), 61), _rand((B, N, Hkv, d), 62)
+    O, L = oracle.attn_fwd_kvcache(q, k, v, [N, N], True, 0.4)
+    O2, L2 = oracle.attn_fwd(q, k, v, True, 0.4)
+    np.testing.assert_allclose(O, O2, atol=1e-13)
+    np.testing.assert_allclose(L, L2, atol=1e-13)
+
+
+def test_kvcache_rows_against_brute_force():
+    """Per-row brute force with Python loops: lengths shorter than the cache,
+    bottom-right causal positions, an empty cache row, GQA mapping."""
+    import math
+    B, Nq, Hq, Hkv, Nc, d, scale = 3, 3, 4, 2, 10, 5, 0.7
+    q, k, v = _rand((B, Nq, Hq, d), 63), _rand((B, Nc, Hkv, d), 64), _rand((B, Nc, Hkv, d), 65)
+    lens = [10, 2, 0]
+    for causal in (False, True):
+        O, L = oracle.attn_fwd_kvcache(q, k, v, lens, causal, scale)
+        for b in range(B):
+            for h in range(Hq):
+                g = h // 2
+                for i in range(Nq):
+                    vis = [j for j in range(lens[b]) if not (causal and j > lens[b] - Nq + i)]
+                    if not vis:
+                        assert np.all(O[b, i, h] == 0) and L[b, h, i] == -np.inf
+                        continue
+                    sc = [scale * sum(q[b, i, h, c] * k[b, j, g, c] for c in range(d)) for j in vis]
+                    den = sum(math.exp(x) for x in sc)
+                    want = [sum(math.exp(x) * v[b, j, g, c] for x, j in zip(sc, vis)) / den for c in range(d)]
+                    np.testing.assert_allclose(O[b, i, h], want, atol=1e-12)
+                    assert abs(L[b, h, i] - math.log(den)) < 1e-12
+
+
+def test_kvcache_split_merge_reproduces_whole_cache():
+    """Split-KV: attention over disjoint key ranges merged by LSE equals
+    attention over the whole cache (the combination the decode path uses)."""
+    B, Nq, Hq, Hkv, Nc, d = 1, 2, 2, 1, 37, 8
+    q, k, v = _rand((B, Nq, Hq, d), 66), _rand((B, Nc, Hkv, d), 67), _rand((B, Nc, Hkv, d), 68)
+    O, L = oracle.attn_fwd_kvcache(q, k, v, [Nc], False, 0.5)
+    outs, lses = [], []
+    for a, e in ((0, 16), (16, 32), (32, 37)):
+        o, l = oracle.attn_fwd_kvcache(q, k[:, a:e], v[:, a:e], [e - a], False, 0.5)
+        outs.append(o)
+        lses.append(l.transpose(0, 2, 1))  # [B,Nq,Hq] to match O's row layout
+    Om, Lm = oracle.merge_partials(outs, lses)
+    np.testing.assert_allclose(Om, O, atol=1e-12)
+    np.testing.assert_allclose(Lm.transpose(0, 2, 1), L, atol=1e-12)
