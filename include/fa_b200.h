@@ -169,6 +169,30 @@ fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const voi
                           int causal, float scale, void* stream);
 
 /*
+ * Decode: Nq new query rows per sequence against a key/value cache (the
+ * KV-cache API of the Dao-AILab repository overview), split over the cache
+ * and combined through the per-split log-sum-exp.
+ *   q [B,Nq,Hq,d] bf16; k_cache/v_cache [B,Ncache,Hkv,d] bf16 (in);
+ *   cache_seqlens: DEVICE int32 [B], valid cache rows L_b per sequence
+ *   (clamped to 0..Ncache); o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] f32 (out).
+ *   Query i is position L_b - Nq + i of its sequence: with causal = 1 it sees
+ *   keys 0 .. L_b - Nq + i, otherwise keys 0 .. L_b - 1. A row that sees no
+ *   key gets O = 0 and LSE = -inf.
+ *   Nq * (Hq/Hkv) <= 16 (FA_ERR_UNSUPPORTED otherwise); d = 64 or 128.
+ *   num_splits >= 1: the cache is cut into that many ranges of whole 128-key
+ *   tiles (fewer if Ncache is short); with more than one range the partial
+ *   results go to `workspace` (DEVICE, 16-byte aligned, at least
+ *   fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) bytes) and a second
+ *   kernel merges them. Bound by HBM bandwidth: the cache is read once.
+ */
+fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
+                           void* o, float* lse, void* workspace, size_t ws_bytes, int B, int Nq, int Hq, int Hkv,
+                           int Ncache, int d, int causal, float scale, int num_splits, void* stream);
+
+/* Workspace bytes of fa_fwd_kvcache (0 when num_splits <= 1). */
+size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_splits);
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (FA_OK if no kernel reported an error since the last
  * call). Returns FA_ERR_CUDA if the synchronisation itself failed.

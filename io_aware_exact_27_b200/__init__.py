@@ -43,6 +43,7 @@ _SIGS = {
     "fa_bwd_varlen": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_get_status": [_P],
     "fa_set_exp_emulation": [_I],
+    "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -51,6 +52,8 @@ for _name, _args in _SIGS.items():
     getattr(_lib, _name).restype = _I
 _lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_size.restype = _Z
+_lib.fa_fwd_kvcache_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+_lib.fa_fwd_kvcache_workspace_size.restype = _Z
 _lib.fa_status_string.argtypes = [_I]
 _lib.fa_status_string.restype = ctypes.c_char_p
 _lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
@@ -121,6 +124,17 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N
     _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                        _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)),
            "fa_bwd")
+
+
+def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_bytes, B, Nq, Hq, Hkv, Ncache, d,
+                   causal, scale, num_splits, stream=None):
+    _check(_lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(o), _ptr(lse),
+                               _ptr(workspace), ws_bytes, B, Nq, Hq, Hkv, Ncache, d, int(causal), float(scale),
+                               int(num_splits), _stream(stream)), "fa_fwd_kvcache")
+
+
+def fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) -> int:
+    return int(_lib.fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits))
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, stream=None):
@@ -234,3 +248,23 @@ def attention_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, causal=F
     fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), cu_seqlens, nseq, max_seqlen, T,
                   Hq, Hkv, d, causal, _default_scale(d, scale), stream)
     return dq, dk, dv
+
+
+def attention_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal=True, scale=None, num_splits=None,
+                          stream=None):
+    """q [B,Nq,Hq,d], caches [B,Ncache,Hkv,d] bf16, cache_seqlens int32 [B] (CUDA)
+    -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] f32). num_splits defaults to enough
+    cache ranges to give every SM about two blocks."""
+    import torch
+    B, Nq, Hq, d = q.shape
+    Ncache, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if num_splits is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = max(1, min((Ncache + 127) // 128, -(-2 * sms // (B * Hkv))))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    ws_bytes = fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, ws, ws_bytes, B, Nq, Hq, Hkv, Ncache, d, causal,
+                   _default_scale(d, scale), num_splits, stream)
+    return o, lse

@@ -11,6 +11,7 @@
 
 #include "../../include/fa_b200.h"
 #include "fa_bwd_kernel.cuh"
+#include "fa_decode_kernel.cuh"
 
 namespace {
 
@@ -34,6 +35,7 @@ struct DeviceState {
   int* status = nullptr;     // device address of g_status_word
   bool fwd_attr[3][6] = {};
   bool bwd_attr[2] = {false, false};
+  bool dec_attr[2] = {false, false};
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -321,6 +323,43 @@ fa_status_t noalloc_scratch_address(void** out) {
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- decode (KV cache)
+size_t dec_part_floats(int B, int Nq, int Hq, int d, int splits) {
+  return static_cast<size_t>(splits) * B * Nq * Hq * (static_cast<size_t>(d) + 1);
+}
+
+template <int D>
+fa_status_t launch_decode(DeviceState* ds, const void* kc, const void* vc, fa::DecArgs a, cudaStream_t stream) {
+  using Smem = fa::DecSmem<D>;
+  auto kern = fa::fa_decode_kernel<D>;
+  const int smem = static_cast<int>(sizeof(Smem)) + 1024;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    bool& done = ds->dec_attr[D == 128 ? 1 : 0];
+    if (!done) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return FA_ERR_CUDA;
+      done = true;
+    }
+  }
+  CUtensorMap tk, tv;
+  fa_status_t st;
+  const int tokens = a.B * a.Ncache;
+  if ((st = encode_rows(&tk, kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_rows(&tv, vc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  a.timeout_ns = g_timeout_ns.load();
+  a.status = ds->status;
+  dim3 grid(a.splits, a.Hkv, a.B);
+  kern<<<grid, fa::kDecThreads, smem, stream>>>(tk, tv, a);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (a.splits > 1) {
+    const long long rows = static_cast<long long>(a.B) * a.Nq * a.Hq;
+    fa::fa_decode_merge_kernel<D><<<static_cast<int>((rows + 7) / 8), 256, 0, stream>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -434,6 +473,53 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   // backward writes every entry the later two read.
   return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, causal, scale,
                 stream);
+}
+
+size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_splits) {
+  if (B <= 0 || Nq <= 0 || Hq <= 0 || d <= 0 || num_splits <= 1) return 0;
+  return dec_part_floats(B, Nq, Hq, d, num_splits) * sizeof(float);
+}
+
+fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
+                           void* o, float* lse, void* workspace, size_t ws_bytes, int B, int Nq, int Hq, int Hkv,
+                           int Ncache, int d, int causal, float scale, int num_splits, void* stream) {
+  if (B < 0 || Nq < 0 || Ncache < 0 || num_splits < 1) return FA_ERR_INVALID_ARG;
+  if (B == 0 || Nq == 0) return FA_OK;
+  fa_status_t st = check_common(q, k_cache, v_cache, o, lse, Hq, Hkv, d, scale);
+  if (st != FA_OK) return st;
+  if (cache_seqlens == nullptr || !aligned(cache_seqlens, 4) || Ncache == 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (Nq * (Hq / Hkv) > fa::kDecRows) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Ncache > INT32_MAX || B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  const int chunk = ((Ncache + num_splits - 1) / num_splits + fa::kDecKeys - 1) / fa::kDecKeys * fa::kDecKeys;
+  const int splits = (Ncache + chunk - 1) / chunk;  // no empty trailing splits
+  if (splits > 1) {
+    if (workspace == nullptr || !aligned(workspace, 16) ||
+        ws_bytes < dec_part_floats(B, Nq, Hq, d, splits) * sizeof(float))
+      return FA_ERR_WORKSPACE;
+  }
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  fa::DecArgs a{};
+  a.q = q;
+  a.cache_seqlens = cache_seqlens;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Nq = Nq;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Ncache = Ncache;
+  a.splits = splits;
+  a.chunk = chunk;
+  a.causal = causal;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  if (splits > 1) {
+    a.part_o = static_cast<float*>(workspace);
+    a.part_lse = a.part_o + static_cast<size_t>(splits) * B * Nq * Hq * d;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_decode<128>(ds, k_cache, v_cache, a, s) : launch_decode<64>(ds, k_cache, v_cache, a, s);
 }
 
 fa_status_t fa_get_status(void* stream) {
