@@ -193,6 +193,15 @@ fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cac
 size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_splits);
 
 /*
+ * Split count fa_fwd_kvcache runs fastest with on the current device for B
+ * sequences, Hkv key/value heads and a cache of Ncache rows: one persistent
+ * CTA per SM streams (sequence, kv head, split) units back to back, and the
+ * count balances the units over the SMs. Returns 1 for non-positive sizes or
+ * when no CUDA device is usable. Not in the pages (a host-side choice).
+ */
+int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache);
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (FA_OK if no kernel reported an error since the last
  * call). Returns FA_ERR_CUDA if the synchronisation itself failed.

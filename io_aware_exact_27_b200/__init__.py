@@ -54,6 +54,8 @@ _lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_size.restype = _Z
 _lib.fa_fwd_kvcache_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.fa_fwd_kvcache_workspace_size.restype = _Z
+_lib.fa_fwd_kvcache_num_splits.argtypes = [_I, _I, _I]
+_lib.fa_fwd_kvcache_num_splits.restype = _I
 _lib.fa_status_string.argtypes = [_I]
 _lib.fa_status_string.restype = ctypes.c_char_p
 _lib.fa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
@@ -135,6 +137,10 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_byt
 
 def fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) -> int:
     return int(_lib.fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits))
+
+
+def fa_fwd_kvcache_num_splits(B, Hkv, Ncache) -> int:
+    return int(_lib.fa_fwd_kvcache_num_splits(B, Hkv, Ncache))
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, stream=None):
@@ -253,14 +259,13 @@ def attention_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, causal=F
 def attention_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal=True, scale=None, num_splits=None,
                           stream=None):
     """q [B,Nq,Hq,d], caches [B,Ncache,Hkv,d] bf16, cache_seqlens int32 [B] (CUDA)
-    -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] f32). num_splits defaults to enough
-    cache ranges to give every SM about two blocks."""
+    -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] f32). num_splits defaults to the
+    library's choice for this device (fa_fwd_kvcache_num_splits)."""
     import torch
     B, Nq, Hq, d = q.shape
     Ncache, Hkv = k_cache.shape[1], k_cache.shape[2]
     if num_splits is None:
-        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
-        num_splits = max(1, min((Ncache + 127) // 128, -(-2 * sms // (B * Hkv))))
+        num_splits = fa_fwd_kvcache_num_splits(B, Hkv, Ncache)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     ws_bytes = fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits)

@@ -80,7 +80,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 // [tokens, heads, d] tensor with 128-row x 64-element (128-byte) boxes, 128B swizzle.
 fa_status_t encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int tokens,
-                        int heads, int d) {
+                        int heads, int d, CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return FA_ERR_CUDA;
   const int box_inner = 128 / elem_bytes;
@@ -91,8 +91,7 @@ fa_status_t encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, 128};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -328,6 +327,23 @@ size_t dec_part_floats(int B, int Nq, int Hq, int d, int splits) {
   return static_cast<size_t>(splits) * B * Nq * Hq * (static_cast<size_t>(d) + 1);
 }
 
+// Query rows of one (batch, kv head) unit: a box of {64 columns, G heads,
+// Nq queries} from q [B*Nq, Hq, d], landing as R = Nq*G rows of 128 bytes
+// (row i*G + g) with the 128-byte swizzle.
+fa_status_t encode_query_rows(CUtensorMap* m, const void* q, int B, int Nq, int Hq, int G, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Hq),
+                        static_cast<cuuint64_t>(B) * static_cast<cuuint64_t>(Nq)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(Hq) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(Nq)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D>
 fa_status_t launch_decode(DeviceState* ds, const void* kc, const void* vc, fa::DecArgs a, cudaStream_t stream) {
   using Smem = fa::DecSmem<D>;
@@ -342,15 +358,19 @@ fa_status_t launch_decode(DeviceState* ds, const void* kc, const void* vc, fa::D
       done = true;
     }
   }
-  CUtensorMap tk, tv;
+  CUtensorMap tq, tk, tv;
   fa_status_t st;
   const int tokens = a.B * a.Ncache;
-  if ((st = encode_rows(&tk, kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
-  if ((st = encode_rows(&tv, vc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D)) != FA_OK) return st;
+  if ((st = encode_query_rows(&tq, a.q, a.B, a.Nq, a.Hq, a.Hq / a.Hkv, D)) != FA_OK) return st;
+  // a head's cache row is D*2 bytes: promote L2 fills to no more than that,
+  // so that a 64-wide head does not drag its neighbour's row in with it
+  const CUtensorMapL2promotion promo = D == 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+  if ((st = encode_rows(&tk, kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D, promo)) != FA_OK) return st;
+  if ((st = encode_rows(&tv, vc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, a.Hkv, D, promo)) != FA_OK) return st;
   a.timeout_ns = g_timeout_ns.load();
   a.status = ds->status;
-  dim3 grid(a.splits, a.Hkv, a.B);
-  kern<<<grid, fa::kDecThreads, smem, stream>>>(tk, tv, a);
+  const int grid = a.num_units < ds->sms ? a.num_units : ds->sms;
+  kern<<<grid, fa::kDecThreads, smem, stream>>>(tq, tk, tv, a);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (a.splits > 1) {
     const long long rows = static_cast<long long>(a.B) * a.Nq * a.Hq;
@@ -358,6 +378,12 @@ fa_status_t launch_decode(DeviceState* ds, const void* kc, const void* vc, fa::D
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
+}
+
+// Keys per split for a requested split count: whole 128-key tiles.
+int dec_chunk_keys(int Ncache, int num_splits) {
+  const int per = (Ncache + num_splits - 1) / num_splits;
+  return (per + fa::kDecKeys - 1) / fa::kDecKeys * fa::kDecKeys;
 }
 
 }  // namespace
@@ -480,6 +506,31 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
   return dec_part_floats(B, Nq, Hq, d, num_splits) * sizeof(float);
 }
 
+int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache) {
+  if (B <= 0 || Hkv <= 0 || Ncache <= 0) return 1;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != FA_OK) return 1;
+  // Each persistent CTA streams its units back to back, so a launch lasts
+  // about (rounds of units) x (tiles per unit + a little per unit): pick the
+  // split count that minimises it.
+  const int tiles = (Ncache + fa::kDecKeys - 1) / fa::kDecKeys;
+  const long long bh = static_cast<long long>(B) * Hkv;
+  double best = 0;
+  int best_s = 1;
+  for (int s = 1; s <= tiles && s <= 256; ++s) {
+    const int chunk = dec_chunk_keys(Ncache, s);
+    const int splits = (Ncache + chunk - 1) / chunk;
+    const int per = chunk / fa::kDecKeys;
+    const long long rounds = (bh * splits + ds->sms - 1) / ds->sms;
+    const double cost = static_cast<double>(rounds) * (per + 0.5) + (splits > 1 ? 0.5 : 0.0);
+    if (s == 1 || cost < best - 1e-9) {
+      best = cost;
+      best_s = splits;
+    }
+  }
+  return best_s;
+}
+
 fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
                            void* o, float* lse, void* workspace, size_t ws_bytes, int B, int Nq, int Hq, int Hkv,
                            int Ncache, int d, int causal, float scale, int num_splits, void* stream) {
@@ -491,8 +542,9 @@ fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cac
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (Nq * (Hq / Hkv) > fa::kDecRows) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * Ncache > INT32_MAX || B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
-  const int chunk = ((Ncache + num_splits - 1) / num_splits + fa::kDecKeys - 1) / fa::kDecKeys * fa::kDecKeys;
+  const int chunk = dec_chunk_keys(Ncache, num_splits);
   const int splits = (Ncache + chunk - 1) / chunk;  // no empty trailing splits
+  if (static_cast<long long>(B) * Hkv * splits > INT32_MAX) return FA_ERR_UNSUPPORTED;
   if (splits > 1) {
     if (workspace == nullptr || !aligned(workspace, 16) ||
         ws_bytes < dec_part_floats(B, Nq, Hq, d, splits) * sizeof(float))
@@ -512,6 +564,7 @@ fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cac
   a.Ncache = Ncache;
   a.splits = splits;
   a.chunk = chunk;
+  a.num_units = B * Hkv * splits;
   a.causal = causal;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   if (splits > 1) {
