@@ -194,12 +194,13 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
 
 /*
  * Split count fa_fwd_kvcache runs fastest with on the current device for B
- * sequences, Hkv key/value heads and a cache of Ncache rows: one persistent
- * CTA per SM streams (sequence, kv head, split) units back to back, and the
- * count balances the units over the SMs. Returns 1 for non-positive sizes or
- * when no CUDA device is usable. Not in the pages (a host-side choice).
+ * sequences, Hkv key/value heads, a cache of Ncache rows and head dim d: one
+ * persistent CTA per SM streams (sequence, kv head, split) units back to back;
+ * the count trades idle SMs against per-unit and merge costs (a launch-time
+ * model with constants measured on B200). Returns 1 for invalid sizes or when
+ * no CUDA device is usable. Not in the pages (a host-side choice).
  */
-int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache);
+int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d);
 
 /*
  * Synchronises `stream`, then returns and clears the device-side status word

@@ -54,7 +54,7 @@ _lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_size.restype = _Z
 _lib.fa_fwd_kvcache_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.fa_fwd_kvcache_workspace_size.restype = _Z
-_lib.fa_fwd_kvcache_num_splits.argtypes = [_I, _I, _I]
+_lib.fa_fwd_kvcache_num_splits.argtypes = [_I, _I, _I, _I]
 _lib.fa_fwd_kvcache_num_splits.restype = _I
 _lib.fa_status_string.argtypes = [_I]
 _lib.fa_status_string.restype = ctypes.c_char_p
@@ -139,8 +139,8 @@ def fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) -> int:
     return int(_lib.fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits))
 
 
-def fa_fwd_kvcache_num_splits(B, Hkv, Ncache) -> int:
-    return int(_lib.fa_fwd_kvcache_num_splits(B, Hkv, Ncache))
+def fa_fwd_kvcache_num_splits(B, Hkv, Ncache, d) -> int:
+    return int(_lib.fa_fwd_kvcache_num_splits(B, Hkv, Ncache, d))
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, stream=None):
@@ -265,7 +265,7 @@ def attention_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal=True, scale
     B, Nq, Hq, d = q.shape
     Ncache, Hkv = k_cache.shape[1], k_cache.shape[2]
     if num_splits is None:
-        num_splits = fa_fwd_kvcache_num_splits(B, Hkv, Ncache)
+        num_splits = fa_fwd_kvcache_num_splits(B, Hkv, Ncache, d)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     ws_bytes = fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits)

@@ -506,24 +506,31 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
   return dec_part_floats(B, Nq, Hq, d, num_splits) * sizeof(float);
 }
 
-int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache) {
-  if (B <= 0 || Hkv <= 0 || Ncache <= 0) return 1;
+int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d) {
+  if (B <= 0 || Hkv <= 0 || Ncache <= 0 || (d != 64 && d != 128)) return 1;
   DeviceState* ds = nullptr;
   if (device_state(&ds) != FA_OK) return 1;
-  // Each persistent CTA streams its units back to back, so a launch lasts
-  // about (rounds of units) x (tiles per unit + a little per unit): pick the
-  // split count that minimises it.
+  // Launch-time model of the decode kernel, its constants measured on B200:
+  // one CTA streams a 128-key tile in about t_tile when HBM is not the limit,
+  // pays about t_unit per (sequence, kv head, split) unit, and the whole cache
+  // cannot stream faster than the HBM rate; more than one split adds the
+  // merge kernel. The persistent CTAs take units round-robin.
+  const double t_tile = d == 128 ? 1.07e-6 : 0.93e-6;
+  const double t_unit = 5e-6, t_merge = 12e-6, hbm_bytes_per_s = 6.4e12;
   const int tiles = (Ncache + fa::kDecKeys - 1) / fa::kDecKeys;
   const long long bh = static_cast<long long>(B) * Hkv;
+  const double t_hbm = 4.0 * static_cast<double>(bh) * Ncache * d / hbm_bytes_per_s;
   double best = 0;
   int best_s = 1;
   for (int s = 1; s <= tiles && s <= 256; ++s) {
     const int chunk = dec_chunk_keys(Ncache, s);
     const int splits = (Ncache + chunk - 1) / chunk;
+    if (splits != s) continue;  // same launch as a smaller count
     const int per = chunk / fa::kDecKeys;
     const long long rounds = (bh * splits + ds->sms - 1) / ds->sms;
-    const double cost = static_cast<double>(rounds) * (per + 0.5) + (splits > 1 ? 0.5 : 0.0);
-    if (s == 1 || cost < best - 1e-9) {
+    const double t_cta = static_cast<double>(rounds) * (per * t_tile + t_unit);
+    const double cost = (t_cta > t_hbm ? t_cta : t_hbm) + (splits > 1 ? t_merge : 0.0);
+    if (s == 1 || cost < best * 0.99) {  // more splits only for a clear gain
       best = cost;
       best_s = splits;
     }

@@ -16,12 +16,16 @@
 // with fp32 accumulators in TMEM. The path streams the cache once: it is
 // bound by HBM, and the tensor cores only keep the CUDA cores free for the
 // softmax. Warp roles of the persistent CTA (one per SM):
-//   warps 0-3  softmax: thread = key of the tile (TMEM lane), 16 row columns;
-//              online softmax with a lazy maximum (base 2, threshold 8),
-//              P^T written to shared memory as the bf16 B operand, and the
-//              unit's epilogue (thread = output column of O^T)
-//   warp 4     TMA producer: Q rows of each unit, K/V tiles through a ring
-//   warp 5     tcgen05.mma issuer
+//   warps 0-7  softmax, two groups of four that take alternate tiles (the
+//              per-tile chain of TMEM load, barrier, exponentials and P store
+//              is latency-bound, so two tiles are kept in flight). Thread =
+//              key of the tile (TMEM lane), 16 row columns; each group keeps
+//              its own lazy running maximum (base 2, threshold 8), row sums
+//              and O^T accumulator, and the unit's epilogue combines the two
+//              exactly, as two key ranges are combined through their LSE.
+//              P^T goes to shared memory as the bf16 B operand.
+//   warp 8     TMA producer: Q rows of each unit, K/V tiles through a ring
+//   warp 9     tcgen05.mma issuer
 // fa_decode_merge_kernel combines the splits' (O_r, LSE_r):
 //   LSE = log sum exp LSE_r,  O = sum exp(LSE_r - LSE) O_r.
 #pragma once
@@ -32,10 +36,11 @@ namespace fa {
 
 constexpr int kDecRows = 16;   // N of both MMAs: max Nq * (Hq/Hkv)
 constexpr int kDecKeys = 128;  // keys per tile (M of the score MMA)
-constexpr int kDecWarpProducer = 4;
-constexpr int kDecWarpMma = 5;
-constexpr int kDecThreads = 192;
-constexpr int kDecBarSoftmax = 1;  // named barrier of the 4 softmax warps
+constexpr int kDecWarpProducer = 8;
+constexpr int kDecWarpMma = 9;
+constexpr int kDecThreads = 320;
+constexpr int kDecBarGroup = 1;    // named barriers 1, 2: the 4 warps of softmax group 0, 1
+constexpr int kDecBarSoftmax = 3;  // named barrier of all 8 softmax warps
 constexpr float kDecTau = 8.f;     // lazy-rescale threshold (log2 units)
 
 struct DecArgs {
@@ -62,13 +67,15 @@ struct DecSmem {
   alignas(1024) uint8_t kv[kStages][2][kTileBytes];    // [slot][K, V]
   alignas(1024) uint8_t q[2][D / 64][kRowBox];         // query rows of a unit, double-buffered
   alignas(1024) uint8_t p[2][2][kRowBox];              // P [16 rows, 128 keys] bf16 (two 64-key atoms), x2
-  float red_m[kDecRows][4];                            // per-warp column maxima
-  float red_l[kDecRows][4];                            // per-warp column sums
+  float red_m[2][kDecRows][4];                         // per group: per-warp column maxima
+  float red_l[2][kDecRows][4];                         // per group: per-warp column sums
+  float xm[2][2][kDecRows], xl[2][2][kDecRows];        // [unit parity][group]: running max, row sums
+  int xn[2][2];                                        // [unit parity][group]: tiles the group took
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t o_full[2], o_empty[2];
-  uint64_t p_full[2], pv_done[2];  // per P buffer
+  uint64_t p_full[2];  // per softmax group (P buffer)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -170,18 +177,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_init(smem_u32(&sm.s_full[i]), 1);
       mbar_init(smem_u32(&sm.s_free[i]), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(&sm.o_full[i]), 1);
-      mbar_init(smem_u32(&sm.o_empty[i]), 4);
+      mbar_init(smem_u32(&sm.o_empty[i]), 8);  // every softmax warp reads both groups' O^T
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&sm.p_full[i]), 4);
-      mbar_init(smem_u32(&sm.pv_done[i]), 1);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&sm.p_full[i]), 4);
     mbar_init(smem_u32(&sm.drain), 1);
     sm.abort = 0;
     fence_barrier_init();
   }
   if (warp == kDecWarpMma) {
-    tmem_alloc(smem_u32(&sm.tmem_base), 64);  // S^T x2, O^T x2, 16 columns each
+    tmem_alloc(smem_u32(&sm.tmem_base), 128);  // S^T per group, O^T per group x 2 units: 16 columns each
     tmem_relinquish();
   }
   if (warp == kDecWarpProducer && lane == 0) {
@@ -250,8 +254,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       constexpr uint32_t kVLbo = D == 128 ? 16384 : 0;
       uint32_t kv_cons = 0, g = 0, nu = 0, npv = 0;
       bool ok = true;
-      bool have_prev = false, prev_first = false, prev_last = false;
+      bool have_prev = false, prev_last = false;
       uint32_t prev_slot = 0, prev_nu = 0;
+      int prev_t = 0;
       auto wait = [&](uint64_t* bar, uint32_t parity, int site) -> bool {
         if (!mbar_wait(smem_u32(bar), parity, abort, a.timeout_ns)) {
           report_error(a.status, kStatusTimeout, site);
@@ -266,15 +271,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (!wait(&sm.p_full[pb], (npv >> 1) & 1, 92)) return false;
         const uint64_t pdesc = smem_desc(smem_u32(sm.p[pb]), 16, 1024, kSwizzle128B);
         const uint32_t ob = prev_nu & 1;
-        if (prev_first && !wait(&sm.o_empty[ob], ((prev_nu >> 1) & 1) ^ 1, 93)) return false;
+        if (prev_t == 0 && !wait(&sm.o_empty[ob], ((prev_nu >> 1) & 1) ^ 1, 93)) return false;
         const uint64_t vdesc = smem_desc(smem_u32(sm.kv[prev_slot][1]), kVLbo, 1024, kSwizzle128B);
-        const uint32_t o_t = tmem + 32 + 16 * ob;
+        const uint32_t o_t = tmem + 32 + 32 * pb + 16 * ob;  // O^T of the tile's group
 #pragma unroll
         for (int kk = 0; kk < kDecKeys / 16; ++kk)
           mma_f16_ss(o_t, vdesc + static_cast<uint64_t>((kk * 2048) >> 4),
                      pdesc + static_cast<uint64_t>(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), idPV,
-                     (kk > 0 || !prev_first) ? 1u : 0u);
-        tc_commit(smem_u32(&sm.pv_done[pb]));
+                     (kk > 0 || prev_t >= 2) ? 1u : 0u);  // a group's first tile of the unit overwrites
         tc_commit(smem_u32(&sm.kv_empty[prev_slot]));
         if (prev_last) tc_commit(smem_u32(&sm.o_full[ob]));
         ++npv;
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           have_prev = true;
           prev_slot = slot;
           prev_nu = nu;
-          prev_first = t == 0;
+          prev_t = t;
           prev_last = t + 1 == w.ntiles;
           ++kv_cons;
           ++g;
@@ -320,11 +324,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_wait(smem_u32(&sm.drain), 0, nullptr, a.timeout_ns);
     }
   } else {
-    // ======================= softmax warps 0-3 =======================
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ======================= softmax warps 0-7 =======================
+    const int grp = warp >> 2;  // group: takes the tiles with global index g, g % 2 == grp
+    const int gtid = tid & 127;  // key of the tile = TMEM lane = output column in the epilogue
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = 16 * grp;
+    const int bar_grp = kDecBarGroup + grp;
     const float cl = a.scale_log2;
     uint32_t g = 0, nu = 0;
-    bool good = true;  // this warp's waits all succeeded (warp-uniform)
+    bool good = true;    // this warp's waits all succeeded (warp-uniform)
+    bool failed = false;  // a barrier of this group saw a failure (group-uniform)
     auto wait = [&](uint64_t* bar, uint32_t parity, int site) {
       const bool w = __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, abort, a.timeout_ns));
       if (!w) {
@@ -338,7 +347,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const DecUnit w = w_next;
       if (u + static_cast<int>(gridDim.x) < a.num_units) w_next = dec_unit(a, u + gridDim.x);
       if (w.ntiles == 0) {
-        dec_write_empty<D>(a, w, tid, G, R);
+        if (grp == 0) dec_write_empty<D>(a, w, gtid, G, R);
         continue;
       }
       // keys below lim_all are visible to every row; causal rows see fewer
@@ -350,20 +359,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         lp[r] = 0.f;
       }
       const uint32_t ob = nu & 1;
-      bool alive = true;
+      const uint32_t o_col = 32 + 32 * grp + 16 * ob;
+      int mine = 0;  // tiles of this unit taken by the group
       for (int t = 0; t < w.ntiles; ++t, ++g) {
-        const uint32_t sb = g & 1;
-        wait(&sm.s_full[sb], (g >> 1) & 1, 97);
+        if ((g & 1) != static_cast<uint32_t>(grp) || failed) continue;
+        wait(&sm.s_full[grp], (g >> 1) & 1, 97);
         float x[kDecRows];
         bool need = false;
-        const int key = w.k_begin + t * kDecKeys + tid;
+        const int key = w.k_begin + t * kDecKeys + gtid;
         if (good) {
           tc_fence_after();
           uint32_t raw[16];
-          tmem_ld16(tmem + lane_off + 16 * sb, raw);
+          tmem_ld16(tmem + lane_off + s_col, raw);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[sb]));
+          if (lane == 0) mbar_arrive(smem_u32(&sm.s_free[grp]));
           if (w.k_begin + (t + 1) * kDecKeys <= lim_all) {
             // every key of the tile is visible to every row
 #pragma unroll
@@ -387,28 +397,39 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             }
           }
         }
-        // the maximum is refreshed only when a score passes it by more than
-        // the threshold (always on the unit's first tile)
-        bool rescale = false;
-        float alpha[kDecRows];
-        if (bar_red_or(need || !good, kDecBarSoftmax, 128)) {
+        // The group's maximum is refreshed only when a score passes it by
+        // more than the threshold (always on the group's first tile). The
+        // group's previous tile (g-2) has finished its P V by now: the score
+        // MMA of tile g was committed after that P V was issued, and a commit
+        // completes only when everything issued before it has. So the P
+        // buffer is free and the group's O^T may be rescaled.
+        if (bar_red_or(need || !good, bar_grp, 128)) {
           if (good) {
             const float cm = warp_colreduce16<true>(x, lane);
-            if ((lane & 1) == 0) sm.red_m[lane >> 1][warp] = cm;
+            if ((lane & 1) == 0) sm.red_m[grp][lane >> 1][warp & 3] = cm;
           }
-          if (!bar_red_and(good, kDecBarSoftmax, 128)) {
-            alive = false;
-            break;
+          if (!bar_red_and(good, bar_grp, 128)) {
+            failed = true;  // skip the rest; the epilogue barrier ends both groups
+            continue;
+          }
+          uint32_t o[16];
+          if (mine > 0) {
+            tc_fence_after();
+            tmem_ld16(tmem + lane_off + o_col, o);
           }
 #pragma unroll
           for (int r = 0; r < kDecRows; ++r) {
-            const float4 c4 = *reinterpret_cast<const float4*>(sm.red_m[r]);
+            const float4 c4 = *reinterpret_cast<const float4*>(sm.red_m[grp][r]);
             const float mn = fmaxf(m[r], fmaxf(fmaxf(c4.x, c4.y), fmaxf(c4.z, c4.w)));
-            alpha[r] = mn == -INFINITY ? 1.f : ex2_approx(m[r] - mn);
-            lp[r] *= alpha[r];
+            const float alpha = mn == -INFINITY ? 1.f : ex2_approx(m[r] - mn);
+            lp[r] *= alpha;
             m[r] = mn;
+            o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha);
           }
-          rescale = t > 0;
+          if (mine > 0) {
+            tmem_st16(tmem + lane_off + o_col, o);
+            tmem_st_wait();
+          }
         }
         uint32_t pbits[kDecRows / 2];  // bf16 pairs: rows 2k (low half), 2k+1 (high half)
         if (good) {
@@ -421,64 +442,74 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             pbits[r / 2] = pack_bf16x2(p0, p1);
           }
         }
-        // P buffer g&1 was last read by the P V of tile g-2; O^T may only be
-        // rescaled once the P V of tile g-1 has finished
-        const uint32_t pb = g & 1;
-        if (rescale) wait(&sm.pv_done[pb ^ 1], ((g - 1) >> 1) & 1, 98);
-        if (g >= 2) wait(&sm.pv_done[pb], ((g >> 1) & 1) ^ 1, 98);
         if (good) {
-          tc_fence_after();
-          if (rescale) {
-            uint32_t o[16];
-            tmem_ld16(tmem + lane_off + 32 + 16 * ob, o);
-#pragma unroll
-            for (int r = 0; r < kDecRows; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
-            tmem_st16(tmem + lane_off + 32 + 16 * ob, o);
-            tmem_st_wait();
-          }
-          uint8_t* pbuf = &sm.p[pb][0][0];
+          uint8_t* pbuf = &sm.p[grp][0][0];
 #pragma unroll
           for (int r = 0; r < kDecRows; ++r)
-            *reinterpret_cast<uint16_t*>(pbuf + dec_p_offset(r, tid)) =
+            *reinterpret_cast<uint16_t*>(pbuf + dec_p_offset(r, gtid)) =
                 static_cast<uint16_t>((r & 1) ? (pbits[r / 2] >> 16) : (pbits[r / 2] & 0xffffu));
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[pb]));
+          if (lane == 0) mbar_arrive(smem_u32(&sm.p_full[grp]));
         }
+        ++mine;
       }
-      if (!alive) break;
-      // ---- epilogue of the unit: l = column sums of the per-key partials
-      if (good) {
-        const float cs = warp_colreduce16<false>(lp, lane);
-        if ((lane & 1) == 0) sm.red_l[lane >> 1][warp] = cs;
+      // ---- epilogue of the unit. Each group: row sums = column sums of the
+      // per-key partials; then the groups swap (max, sums, tile counts).
+      const int par = nu & 1;
+      if (!failed && mine > 0) {
+        if (good) {
+          const float cs = warp_colreduce16<false>(lp, lane);
+          if ((lane & 1) == 0) sm.red_l[grp][lane >> 1][warp & 3] = cs;
+        }
+        if (!bar_red_and(good, bar_grp, 128)) failed = true;
       }
-      if (!bar_red_and(good, kDecBarSoftmax, 128)) break;
+      if (gtid == 0) {
+#pragma unroll
+        for (int r = 0; r < kDecRows; ++r) {
+          const float4 c4 = *reinterpret_cast<const float4*>(sm.red_l[grp][r]);
+          sm.xm[par][grp][r] = m[r];
+          sm.xl[par][grp][r] = mine > 0 ? (c4.x + c4.y) + (c4.z + c4.w) : 0.f;
+        }
+        sm.xn[par][grp] = mine;
+      }
+      if (!bar_red_and(good && !failed, kDecBarSoftmax, 256)) break;
+      const int n0 = sm.xn[par][0], n1 = sm.xn[par][1];
       wait(&sm.o_full[ob], (nu >> 1) & 1, 99);
       if (good) {
+        // this group writes rows 8*grp .. 8*grp+7: columns 8*grp.. of both O^T
         tc_fence_after();
-        uint32_t o[16];
-        tmem_ld16(tmem + lane_off + 32 + 16 * ob, o);
+        uint32_t o0[8], o1[8];
+        if (n0 > 0) tmem_ld8(tmem + lane_off + 32 + 16 * ob + 8 * grp, o0);
+        if (n1 > 0) tmem_ld8(tmem + lane_off + 64 + 16 * ob + 8 * grp, o1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.o_empty[ob]));
         const size_t ps = static_cast<size_t>(w.split) * a.B * a.Nq * a.Hq;
 #pragma unroll
-        for (int r = 0; r < kDecRows; ++r) {
+        for (int c = 0; c < 8; ++c) {
+          const int r = 8 * grp + c;
           if (r >= R) continue;
-          const float4 c4 = *reinterpret_cast<const float4*>(sm.red_l[r]);
-          const float l = (c4.x + c4.y) + (c4.z + c4.w);
+          const float m0 = sm.xm[par][0][r], m1 = sm.xm[par][1][r];
+          const float mm = fmaxf(m0, m1);
+          const float w0 = (n0 > 0 && m0 != -INFINITY) ? ex2_approx(m0 - mm) : 0.f;
+          const float w1 = (n1 > 0 && m1 != -INFINITY) ? ex2_approx(m1 - mm) : 0.f;
+          const float l = w0 * sm.xl[par][0][r] + w1 * sm.xl[par][1][r];
+          float acc = 0.f;
+          if (w0 != 0.f) acc = w0 * __uint_as_float(o0[c]);
+          if (w1 != 0.f) acc = fmaf(w1, __uint_as_float(o1[c]), acc);
           const int i = r / G, hq = w.hk * G + (r - i * G);
           const size_t orow = (static_cast<size_t>(w.b) * a.Nq + i) * a.Hq + hq;
           const size_t li = (static_cast<size_t>(w.b) * a.Hq + hq) * a.Nq + i;
-          const float val = l > 0.f ? __uint_as_float(o[r]) / l : 0.f;
-          const float lse = l > 0.f ? m[r] * 0.6931471805599453f + logf(l) : -INFINITY;
+          const float val = l > 0.f ? acc / l : 0.f;
+          const float lse = l > 0.f ? mm * 0.6931471805599453f + logf(l) : -INFINITY;
           if (a.splits == 1) {
-            if (tid < D) reinterpret_cast<__nv_bfloat16*>(a.o)[orow * D + tid] = __float2bfloat16_rn(val);
-            if (tid == 0) a.lse[li] = lse;
+            if (gtid < D) reinterpret_cast<__nv_bfloat16*>(a.o)[orow * D + gtid] = __float2bfloat16_rn(val);
+            if (gtid == 0) a.lse[li] = lse;
           } else {
-            if (tid < D) a.part_o[(ps + orow) * D + tid] = val;
-            if (tid == 0) a.part_lse[ps + li] = lse;
+            if (gtid < D) a.part_o[(ps + orow) * D + gtid] = val;
+            if (gtid == 0) a.part_lse[ps + li] = lse;
           }
         }
       }
@@ -500,7 +531,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == kDecWarpMma) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, 128);
   }
 }
 
