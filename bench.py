@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
+    ap.add_argument("--workload", default="attention", choices=["attention", "decode"],
+                    help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read")
+    ap.add_argument("--decode-shape", default="16,1,32,8,16384,128",
+                    help="B,Nq,Hq,Hkv,Ncache,d of the decode workload")
     args = ap.parse_args()
     if args.shape:
         B, Hq, Hkv, N, d, c = (int(x) for x in args.shape.split(","))
@@ -386,8 +390,191 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------- decode workload
+
+DEC_METRIC = "decode against a KV cache: GB/s of cache read (HBM-bound)"
+
+
+def decode_shape(args):
+    B, Nq, Hq, Hkv, Nc, d = (int(x) for x in args.decode_shape.split(","))
+    cfg = {"workload": f"bf16 causal decode, B={B} Nq={Nq} Hq={Hq} Hkv={Hkv} Ncache={Nc} (full caches) d={d}",
+           "B": B, "Nq": Nq, "Hq": Hq, "Hkv": Hkv, "Ncache": Nc, "d": d, "causal": True}
+    # algorithmic bytes of one step: the K and V cache rows read once, the
+    # query rows read and the output rows written (bf16), LSE written (fp32)
+    byts = 2 * B * Nc * Hkv * d * 2 + 2 * B * Nq * Hq * d * 2 + B * Hq * Nq * 4
+    return B, Nq, Hq, Hkv, Nc, d, cfg, byts
+
+
+def decode_oracle_sample(args, budget_s):
+    """Times the oracle on whole sequences of the decode workload until
+    `budget_s` is spent; returns (GB/s of cache, sequences, seconds, cores)."""
+    import numpy as np
+    import oracle
+    B, Nq, Hq, Hkv, Nc, d, cfg, byts = decode_shape(args)
+    rng = np.random.default_rng(0)
+    done, el, t_start = 0, 0.0, time.perf_counter()
+    while done < B:
+        q = rng.standard_normal((1, Nq, Hq, d), dtype=np.float32)
+        k = rng.standard_normal((1, Nc, Hkv, d), dtype=np.float32)
+        v = rng.standard_normal((1, Nc, Hkv, d), dtype=np.float32)
+        t1 = time.perf_counter()
+        oracle.attn_fwd_kvcache(q, k, v, np.array([Nc]), True, 1.0 / math.sqrt(d))
+        el += time.perf_counter() - t1  # the oracle's time only, not the input draw
+        done += 1
+        if time.perf_counter() - t_start >= budget_s:
+            break
+    return byts / B * done / el / 1e9, done, el, os.cpu_count()
+
+
+def run_decode_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    B, Nq, Hq, Hkv, Nc, d, cfg, byts = decode_shape(args)
+    per_step_budget = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = decode_oracle_sample(args, per_step_budget)
+        if i >= args.warmup:
+            vals.append(r)
+    gbs = sum(v[0] for v in vals) / len(vals)
+    ms = sum(v[2] for v in vals) / len(vals) * 1e3
+    sample = f"{vals[-1][1]} of {B} sequences per step, fp64 numpy (input draw not timed)"
+    line = {"metric": DEC_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": dict(cfg, parallelism=f"replicas{args.gpus}", l2="n/a (CPU)"),
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": vals[-1][3], "kind": "oracle", "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args):
+    import torch
+    world, rank, local = dist_setup(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    import synth
+    B, Nq, Hq, Hkv, Nc, d, cfg, byts = decode_shape(args)
+    scale = 1.0 / math.sqrt(d)
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank)
+    # the cache is resident state of the decoder (drawn on the device); the
+    # step's inputs are the new query rows and the cache lengths
+    kc = torch.randn((B, Nc, Hkv, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((B, Nc, Hkv, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    import numpy as np
+    q_h = synth.to_bf16(synth.normal_f32(np.random.default_rng(rank), (B, Nq, Hq, d)))
+    lens_h = torch.full((B,), Nc, dtype=torch.int32)
+    q, lens = q_h.to(dev), lens_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+    splits = fa.fa_fwd_kvcache_num_splits(B, Hkv, Nc, d)
+    ws_bytes = fa.fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, splits)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def step():
+        fa.fa_fwd_kvcache(q, kc, vc, lens, o, lse, ws, ws_bytes, B, Nq, Hq, Hkv, Nc, d, 1, scale, splits, sptr)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+    # The cache (B*Ncache*Hkv*d*4 bytes) is far larger than L2: steps run back
+    # to back without a flush; events bracket every step.
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(dev)
+    st = fa.fa_get_status(sptr)
+    if st != fa.FA_OK:
+        raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
+    tot_ms = ev[0].elapsed_time(ev[-1])
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms_per_step = tot_ms / args.steps
+    value = byts * world * args.steps / (tot_ms * 1e-3) / 1e9
+    pk = peaks()
+    per_kernel = byts / (ms_per_step * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "fa_decode_kernel" + (" + fa_decode_merge_kernel" if splits > 1 else ""),
+                "achieved": per_kernel, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": per_kernel / pk["hbm_gbs"],
+                "traffic": traffic_for("fa_decode_kernel"), "peak_source": f"{pk['source']} HBM copy",
+                "bytes_per_launch": byts, "num_splits": splits}
+    e2e = None
+    if args.e2e_steps > 0:
+        q_pin, lens_pin = q_h.pin_memory(), lens_h.pin_memory()
+        o_pin = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_pin = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            q.copy_(q_pin, non_blocking=True)
+            lens.copy_(lens_pin, non_blocking=True)
+            step()
+            o_pin.copy_(o, non_blocking=True)
+            lse_pin.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": byts * world * args.e2e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": q_pin.numel() * 2 + lens_pin.numel() * 4,
+               "d2h_bytes_per_step": o_pin.numel() * 2 + lse_pin.numel() * 4,
+               "note": "the KV cache is resident decoder state; the step's inputs are q and the cache lengths"}
+    cpu = None
+    if rank == 0 and world == 1:
+        gbs, seqs, el, cores = decode_oracle_sample(args, args.cpu_budget_s)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{seqs} of {B} sequences of the workload, fp64 numpy, {el:.1f} s"}
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg.update({"parallelism": f"dp{world}" if world > 1 else "single",
+                "l2": "inputs larger than L2 (cache %.2f GB), no flush" % (2 * B * Nc * Hkv * d * 2 / 1e9),
+                "global_batch": B * world})
+    line = {"metric": DEC_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": args.steps * (2 if splits > 1 else 1)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "decode":
+        return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
