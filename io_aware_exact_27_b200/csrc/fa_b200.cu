@@ -219,10 +219,12 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   if ((st = encode_rows(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hq, D)) != FA_OK) return st;
   a.timeout_ns = g_timeout_ns.load();
   a.status = ds->status;
-  // D and LSE in base 2 (one warp per row, 8 warps per block)
+  // D and LSE in base 2: 8 warps per block, each warp kPrePasses x 32/(D/8)
+  // entries per pass; at most 8 resident blocks per SM
   const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
-  long long pre_blocks = (rows + 7) / 8;
-  if (pre_blocks > static_cast<long long>(ds->sms) * 32) pre_blocks = static_cast<long long>(ds->sms) * 32;
+  const long long per_block = 8LL * (32 / (D / 8)) * fa::kPrePasses;
+  long long pre_blocks = (rows + per_block - 1) / per_block;
+  if (pre_blocks > static_cast<long long>(ds->sms) * 8) pre_blocks = static_cast<long long>(ds->sms) * 8;
   if (parts & FA_BWD_PREPARE) {
     fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;

@@ -63,67 +63,82 @@ struct BwdArgs {
 // of its sequence.
 __device__ __forceinline__ int ws_offset(int tok0, int seq) { return ((tok0 + 3) & ~3) + 4 * seq; }
 
-// One warp per workspace entry (head, i): finds the sequence holding entry i
-// (binary search over the sequence starts), then D = dot(dO, O) in fp32 and
-// the base-2 LSE of that token, or the filler values.
+// Workspace entry r = (head h, index i) -> the token it holds, or -1 for a
+// gap / trailing filler entry: the last sequence whose block starts at or
+// before i (binary search over the sequence starts).
+__device__ __forceinline__ int pre_token(const BwdArgs& a, int i, int& seq, int& row) {
+  int lo = 0, hi = a.nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + mid) : mid * a.N;
+    if (ws_offset(t0, mid) <= i) lo = mid; else hi = mid - 1;
+  }
+  const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + lo) : lo * a.N;
+  const int n = a.cu_seqlens ? __ldg(a.cu_seqlens + lo + 1) - t0 : a.N;
+  seq = lo;
+  row = i - ws_offset(t0, lo);
+  return (row < 0 || row >= n) ? -1 : t0 + row;
+}
+
+// D = dot(dO, O) in fp32 and the base-2 LSE for every workspace entry, or the
+// filler values. D/8 lanes share an entry (16-byte loads, 8 elements per
+// lane); a warp takes 32/(D/8) entries per pass and issues the loads of kPrePasses
+// passes before reducing any, so that each warp keeps several rows in flight.
+constexpr int kPrePasses = 4;
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
+  constexpr int LPR = D / 8;     // lanes per entry
+  constexpr int EPW = 32 / LPR;  // entries per warp per pass
   const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, sl = lane % LPR;
   const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
   const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  constexpr int PER = D / 32;  // elements per lane
-  for (long long r = w0; r < rows; r += nw) {
-    const int h = static_cast<int>(r / a.ws_stride);
-    const int i = static_cast<int>(r - static_cast<long long>(h) * a.ws_stride);
-    // last sequence whose workspace block starts at or before i
-    int lo = 0, hi = a.nseq - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + mid) : mid * a.N;
-      if (ws_offset(t0, mid) <= i) lo = mid; else hi = mid - 1;
-    }
-    const int t0 = a.cu_seqlens ? __ldg(a.cu_seqlens + lo) : lo * a.N;
-    const int n = a.cu_seqlens ? __ldg(a.cu_seqlens + lo + 1) - t0 : a.N;
-    const int row = i - ws_offset(t0, lo);
-    if (row < 0 || row >= n) {
-      if (lane == 0) {
-        a.lse2[r] = INFINITY;
-        a.dvec[r] = 0.f;
-      }
-      continue;
-    }
-    const int tok = t0 + row;
-    const size_t base = (static_cast<size_t>(tok) * a.Hq + h) * D + lane * PER;
-    const __nv_bfloat16* op = reinterpret_cast<const __nv_bfloat16*>(a.o) + base;
-    const __nv_bfloat16* gp = reinterpret_cast<const __nv_bfloat16*>(a.dout) + base;
-    float acc = 0.f;
-    if constexpr (PER == 4) {
-      const uint2 ov = *reinterpret_cast<const uint2*>(op);
-      const uint2 gv = *reinterpret_cast<const uint2*>(gp);
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+  for (long long base = w0 * EPW * kPrePasses; base < rows; base += nw * EPW * kPrePasses) {
+    uint4 ov[kPrePasses], gv[kPrePasses];
+    float lv[kPrePasses];
+    int tok[kPrePasses];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float2 x = __bfloat1622float2(o2[t]);
-        const float2 y = __bfloat1622float2(g2[t]);
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
+    for (int u = 0; u < kPrePasses; ++u) {
+      const long long r = base + u * EPW + sub;
+      tok[u] = -1;
+      lv[u] = 0.f;
+      if (r < rows) {
+        const int h = static_cast<int>(r / a.ws_stride);
+        const int i = static_cast<int>(r - static_cast<long long>(h) * a.ws_stride);
+        int seq, row;
+        tok[u] = pre_token(a, i, seq, row);
+        if (tok[u] >= 0) {
+          const size_t off = (static_cast<size_t>(tok[u]) * a.Hq + h) * D + sl * 8;
+          ov[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + off));
+          gv[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dout) + off));
+          const size_t li = a.cu_seqlens ? static_cast<size_t>(h) * a.lse_head_stride + tok[u]
+                                         : (static_cast<size_t>(seq) * a.Hq + h) * a.lse_head_stride + row;
+          if (sl == 0) lv[u] = __ldg(a.lse + li);
+        }
       }
-    } else {
-      const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(op);
-      const __nv_bfloat162 g2 = *reinterpret_cast<const __nv_bfloat162*>(gp);
-      const float2 x = __bfloat1622float2(o2);
-      const float2 y = __bfloat1622float2(g2);
-      acc = fmaf(x.x, y.x, x.y * y.y);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      const size_t li = a.cu_seqlens ? static_cast<size_t>(h) * a.lse_head_stride + tok
-                                     : (static_cast<size_t>(lo) * a.Hq + h) * a.lse_head_stride + row;
-      a.lse2[r] = a.lse[li] * kLog2e;
-      a.dvec[r] = acc;
+    for (int u = 0; u < kPrePasses; ++u) {
+      float acc = 0.f;
+      if (tok[u] >= 0) {
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[u]);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[u]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 x = __bfloat1622float2(o2[t]);
+          const float2 y = __bfloat1622float2(g2[t]);
+          acc = fmaf(x.x, y.x, acc);
+          acc = fmaf(x.y, y.y, acc);
+        }
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const long long r = base + u * EPW + sub;
+      if (sl == 0 && r < rows) {
+        a.lse2[r] = tok[u] >= 0 ? lv[u] * kLog2e : INFINITY;
+        a.dvec[r] = tok[u] >= 0 ? acc : 0.f;
+      }
     }
   }
 }
