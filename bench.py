@@ -49,8 +49,12 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
-    ap.add_argument("--workload", default="attention", choices=["attention", "decode"],
-                    help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read")
+    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring"],
+                    help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
+                         "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated)")
+    ap.add_argument("--ring-shape", default="1,32,8,16384,128",
+                    help="B,Hq,Hkv,N,d of the ring workload (causal; N split over the ring)")
+    ap.add_argument("--ring-ranks", type=int, default=4, help="ranks emulated on one GPU (--gpus 1)")
     ap.add_argument("--decode-shape", default="16,1,32,8,16384,128",
                     help="B,Nq,Hq,Hkv,Ncache,d of the decode workload")
     args = ap.parse_args()
@@ -571,8 +575,218 @@ def run_decode(args):
     return 0
 
 
+# ----------------------------------------------------------------- ring workload
+
+RING_METRIC = "context-parallel ring attention forward TFLOP/s (bf16, causal)"
+
+
+def run_ring(args):
+    import torch
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_ring_reference(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    from io_aware_exact_27_b200 import ring as rg
+    import synth
+    B, Hq, Hkv, N, d = (int(x) for x in args.ring_shape.split(","))
+    R = world if world > 1 else args.ring_ranks
+    n = N // R
+    if n * R != N:
+        raise SystemExit("N must split evenly over the ring")
+    scale = 1.0 / math.sqrt(d)
+    # this process's ranks: its own one (NCCL ring) or all R (emulated)
+    mine = [rank] if world > 1 else list(range(R))
+    q_h, k_h, v_h = synth.qkv_bf16(0, B, N, Hq, Hkv, d)
+    sh = lambda t, r: t[:, r * n:(r + 1) * n].contiguous()  # noqa: E731
+    qs = {r: sh(q_h, r).to(dev) for r in range(R)}
+    ks = {r: sh(k_h, r).to(dev) for r in range(R)}
+    vs = {r: sh(v_h, r).to(dev) for r in range(R)}
+    stream = torch.cuda.current_stream(dev)
+    rec = []  # (start, end, flops) of every forward-kernel launch of a timed step
+    recm = []  # (start, end) of every merge step (a launch for ranks with more than one block)
+    timing = {"on": False}
+
+    def rank_fns(r):
+        g = rg._gpu_rank(qs[r], r, R, True, scale)
+
+        def blk(qq, kk, vv, c):
+            if timing["on"]:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            out = g.block(qq, kk, vv, c)
+            if timing["on"]:
+                e1.record(stream)
+                rec.append((e0, e1, fwd_flops(B, Hq, n, d, c)))
+            return out
+
+        def merge(o_t, lse_t, first, last):
+            if timing["on"]:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            out = g.merge(o_t, lse_t, first, last)
+            if timing["on"]:
+                e1.record(stream)
+                recm.append((e0, e1))
+            return out
+        return blk, merge
+
+    def step():
+        res = []
+        for r in mine:
+            if world > 1:
+                blocks = rg.ring_exchange(ks[r], vs[r])
+            else:
+                blocks = (((r - t) % R, ks[(r - t) % R], vs[(r - t) % R]) for t in range(R))
+            blk, merge = rank_fns(r)
+            res.append(rg.ring_forward(qs[r], blocks, r, R, True, blk, merge))
+        return res
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status() != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    e_beg, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    timing["on"] = True
+    with ClockSampler(local) as clk:
+        e_beg.record(stream)
+        for _ in range(args.steps):
+            step()
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+    timing["on"] = False
+    tot_ms = e_beg.elapsed_time(e_end)
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    f_job = fwd_flops(B, Hq, N, d, True)  # the whole sequence's causal attention
+    value = f_job * args.steps / (tot_ms * 1e-3) / 1e12
+    k_ms = sum(a.elapsed_time(b) for a, b, _ in rec)
+    k_fl = sum(f for _, _, f in rec)
+    m_ms = sum(a.elapsed_time(b) for a, b in recm)
+    pk = peaks()
+    achieved = k_fl / (k_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel", "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "peak_source": f"{pk['source']} bf16 burst (cuBLAS)",
+                "launches": len(rec), "kernel_ms_per_step": k_ms / args.steps,
+                "merge_ms_per_step": m_ms / args.steps,
+                "note": "per-launch flops: a full n x n block 4*B*Hq*n^2*d, the causal diagonal block half of it"}
+    clocks = clk.summary()
+    # end to end: this process's shards copied in from pinned host memory,
+    # its O and LSE copied out, every step
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = {r: [sh(t, r).pin_memory() for t in (q_h, k_h, v_h)] for r in mine}
+        outs_h = {r: (torch.empty((B, n, Hq, d), dtype=torch.bfloat16).pin_memory(),
+                      torch.empty((B, Hq, n), dtype=torch.float32).pin_memory()) for r in mine}
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for r in mine:
+                qs[r].copy_(pin[r][0], non_blocking=True)
+                ks[r].copy_(pin[r][1], non_blocking=True)
+                vs[r].copy_(pin[r][2], non_blocking=True)
+            res = step()
+            for r, (o_r, l_r) in zip(mine, res):
+                outs_h[r][0].copy_(o_r, non_blocking=True)
+                outs_h[r][1].copy_(l_r, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(x.numel() * x.element_size() for r in mine for x in pin[r])
+        d2h = sum(x.numel() * x.element_size() for r in mine for x in outs_h[r])
+        e2e = {"value": f_job * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, rows, el, cores = ring_oracle_sample(args, args.cpu_budget_s)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} query rows of head 0, fp64 numpy, {el:.1f} s"}
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = {"workload": f"bf16 causal ring attention forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}, "
+                       f"{R} ranks of {n} tokens" + (" (emulated on one GPU)" if world == 1 else ""),
+           "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "ring_ranks": R,
+           "parallelism": f"cp{world}" if world > 1 else f"cp{R} emulated", "l2": "no flush (whole-job timing)"}
+    line = {"metric": RING_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": len(rec) + len(recm)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def ring_oracle_sample(args, budget_s):
+    """The oracle on sampled query rows of the ring workload (full sequence)."""
+    import numpy as np
+    import oracle
+    import synth
+    B, Hq, Hkv, N, d = (int(x) for x in args.ring_shape.split(","))
+    q, k, v = synth.qkv_bf16(0, 1, N, Hq, Hkv, d)
+    rng = np.random.default_rng(2)
+    done, el = 0, 0.0
+    flops = 0.0
+    while el < budget_s and done < N:
+        rows = np.sort(rng.choice(N, size=64, replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_fwd_rows(q[:, :, :1], k[:, :, :1], v[:, :, :1], True, 1 / math.sqrt(d), rows[None, :])
+        el += time.perf_counter() - t0
+        flops += float(sum(4.0 * (r + 1) * d for r in rows))
+        done += 64
+    return flops / el / 1e12, done, el, os.cpu_count()
+
+
+def run_ring_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    per = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+    vals = [ring_oracle_sample(args, per) for _ in range(args.warmup + args.steps)][args.warmup:]
+    tf = sum(v[0] for v in vals) / len(vals)
+    B, Hq, Hkv, N, d = (int(x) for x in args.ring_shape.split(","))
+    line = {"metric": RING_METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sum(v[2] for v in vals) / len(vals) * 1e3,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"bf16 causal ring attention forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}",
+                       "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+                             "sample": f"{vals[-1][1]} query rows of head 0 per step, fp64 numpy"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "ring":
+        return run_ring(args)
     if args.workload == "decode":
         return run_decode_reference(args) if args.impl == "reference" else run_decode(args)
     if args.impl == "reference":

@@ -203,6 +203,24 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
 int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d);
 
 /*
+ * Merge of attention partials over disjoint key sets (the multi-GPU variants
+ * of the topic page "Flash Attention and Efficient Transformer Mechanisms";
+ * used by context-parallel ring attention): partial t is exact attention of
+ * the same query rows over key shard t, normalised by its own softmax sum, as
+ * fa_fwd writes it; over all shards
+ *   lse = log sum_t exp lse_t,   o = sum_t exp(lse_t - lse) o_t.
+ *   o_parts   DEVICE bf16 [nparts][B,N,H,d], 16-byte aligned (in);
+ *   lse_parts DEVICE fp32 [nparts][B,H,N] natural log (in; -inf for a row of a
+ *             partial that saw no key);
+ *   o DEVICE bf16 [B,N,H,d], 16-byte aligned; lse DEVICE fp32 [B,H,N] (out).
+ *   nparts >= 1; d = 64 or 128. The sums run in fp32. One HBM-bound kernel
+ *   on `stream`.
+ */
+fa_status_t fa_attn_merge(const void* o_parts, const float* lse_parts, int nparts, void* o, float* lse, int B, int N,
+                          int H, int d, void* stream);
+
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (FA_OK if no kernel reported an error since the last
  * call). Returns FA_ERR_CUDA if the synchronisation itself failed.

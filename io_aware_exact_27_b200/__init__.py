@@ -44,6 +44,7 @@ _SIGS = {
     "fa_get_status": [_P],
     "fa_set_exp_emulation": [_I],
     "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
+    "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -133,6 +134,11 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_byt
     _check(_lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(o), _ptr(lse),
                                _ptr(workspace), ws_bytes, B, Nq, Hq, Hkv, Ncache, d, int(causal), float(scale),
                                int(num_splits), _stream(stream)), "fa_fwd_kvcache")
+
+
+def fa_attn_merge(o_parts, lse_parts, nparts, o, lse, B, N, H, d, stream=None):
+    _check(_lib.fa_attn_merge(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, N, H, d,
+                              _stream(stream)), "fa_attn_merge")
 
 
 def fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) -> int:

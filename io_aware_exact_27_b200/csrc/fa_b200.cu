@@ -12,6 +12,7 @@
 #include "../../include/fa_b200.h"
 #include "fa_bwd_kernel.cuh"
 #include "fa_decode_kernel.cuh"
+#include "fa_merge_kernel.cuh"
 
 namespace {
 
@@ -582,6 +583,34 @@ fa_status_t fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cac
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_decode<128>(ds, k_cache, v_cache, a, s) : launch_decode<64>(ds, k_cache, v_cache, a, s);
+}
+
+fa_status_t fa_attn_merge(const void* o_parts, const float* lse_parts, int nparts, void* o, float* lse, int B, int N,
+                          int H, int d, void* stream) {
+  if (B < 0 || N < 0 || H <= 0 || nparts < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!o_parts || !lse_parts || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 16) || !aligned(o, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  fa::MergeArgs a{};
+  a.o_parts = o_parts;
+  a.lse_parts = lse_parts;
+  a.o = o;
+  a.lse = lse;
+  a.rows = static_cast<long long>(B) * N * H;
+  a.N = N;
+  a.H = H;
+  a.nparts = nparts;
+  const long long rows_per_block = 8LL * (32 / (d / 8));  // 8 warps, 32/(d/8) rows each
+  const long long blocks = (a.rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    fa::fa_merge_kernel<128><<<static_cast<int>(blocks), 256, 0, s>>>(a);
+  else
+    fa::fa_merge_kernel<64><<<static_cast<int>(blocks), 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status_t fa_get_status(void* stream) {

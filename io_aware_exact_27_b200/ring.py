@@ -1,0 +1,170 @@
+"""Context-parallel ring attention (forward) over torch.distributed ranks.
+
+The topic page "Flash Attention and Efficient Transformer Mechanisms" (opening
+paragraph) says the method extends to multi-GPU settings for very long
+sequences; the Dao-AILab repository overview (training sub-package) names
+sequence parallelism. Neither gives an algorithm; this module takes the plain
+one (a reading): every rank holds one contiguous shard of the sequence, the
+key/value shards travel once around the ring, and each rank folds the exact
+attention of its query rows over every shard it sees into a running result
+through the log-sum-exp merge of disjoint key sets.
+
+Rank r of R holds tokens [r*n, (r+1)*n) of every sequence (n = N/R) of Q, K
+and V, laid out [B, n, H, d]. At hop t it holds the K/V shard of rank
+src = (r - t) mod R and computes, with the single-GPU forward kernel:
+  * src < r, or no causal mask: every key precedes every query: full block;
+  * src == r: the shard's own keys: causal within the block;
+  * src > r with the causal mask: every key follows every query: skipped.
+While a block is computed the shard moves one hop on (NCCL send to r+1,
+receive from r-1 into a second buffer). Each block's bf16 (O_t, LSE_t) goes
+to its own slot; after the last block `fa_attn_merge` combines the slots in
+fp32 (one pass over them).
+
+Only the exchange of K/V shards crosses GPUs; the arithmetic of every step runs
+in the library's kernels. The contiguous sharding gives causal ranks unequal
+work (rank r computes r + 1 blocks).
+"""
+
+from __future__ import annotations
+
+import math
+
+
+def ring_block_mode(rank: int, src: int, causal: bool) -> str:
+    """How rank `rank`'s query shard attends the key shard of rank `src`."""
+    if not causal or src < rank:
+        return "full"
+    if src == rank:
+        return "causal"
+    return "skip"
+
+
+def ring_schedule(rank: int, world: int, causal: bool):
+    """[(hop, source rank of the K/V shard held at that hop, mode)] for one rank."""
+    return [(t, (rank - t) % world, ring_block_mode(rank, (rank - t) % world, causal)) for t in range(world)]
+
+
+def ring_forward(q, kv_blocks, rank: int, world: int, causal: bool, block_attention, merge):
+    """Transport-agnostic core of the ring.
+
+    kv_blocks yields (src, k, v) in hop order; block_attention(q, k, v,
+    causal) returns (O_t, LSE_t) of one block; merge(o_t, lse_t, first, last)
+    folds it into the running result and returns that result after the last
+    block. Blocks in "skip" mode are not computed; the caller's merge sees
+    first=True on the first computed block and last=True on the last one.
+    """
+    sched = ring_schedule(rank, world, causal)
+    todo = [t for t, _, mode in sched if mode != "skip"]
+    last_t = todo[-1]
+    out = None
+    first = True
+    for t, (src, k, v) in enumerate(kv_blocks):
+        if src != sched[t][1]:
+            raise RuntimeError(f"ring order broken: hop {t} holds shard {src}, expected {sched[t][1]}")
+        mode = sched[t][2]
+        if mode != "skip":
+            o_t, lse_t = block_attention(q, k, v, mode == "causal")
+            out = merge(o_t, lse_t, first, t == last_t)
+            first = False
+    return out
+
+
+def ring_exchange(k, v, group=None):
+    """Yields (src, k, v) for hops 0..R-1 of the ring; the next shard's
+    transfer (send to rank+1, receive from rank-1, both K and V) runs while
+    the caller works on the current one. Works with any torch.distributed
+    backend that has point-to-point ops (NCCL on GPUs, gloo on CPU)."""
+    import torch
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    nxt = dist.get_global_rank(group, (r + 1) % R) if group is not None else (r + 1) % R
+    prv = dist.get_global_rank(group, (r - 1) % R) if group is not None else (r - 1) % R
+    cur = (k, v)
+    spare = (torch.empty_like(k), torch.empty_like(v)) if R > 1 else None
+    for t in range(R):
+        reqs = []
+        if t + 1 < R:
+            ops = [dist.P2POp(dist.isend, cur[0], nxt, group), dist.P2POp(dist.isend, cur[1], nxt, group),
+                   dist.P2POp(dist.irecv, spare[0], prv, group), dist.P2POp(dist.irecv, spare[1], prv, group)]
+            reqs = dist.batch_isend_irecv(ops)
+        yield (r - t) % R, cur[0], cur[1]
+        for req in reqs:
+            req.wait()
+        if t + 1 < R:
+            cur, spare = spare, cur
+
+
+class _GpuRank:
+    """The GPU side of one rank's ring: each computed block writes its bf16
+    (O_t, LSE_t) into its own slot, and after the last block one merge kernel
+    combines the slots (a rank with a single block returns it as is)."""
+
+    def __init__(self, q_shape, nblocks, scale, device):
+        import torch
+        B, n, H, d = q_shape
+        self.shape = (B, n, H, d)
+        self.scale = scale
+        self.nblocks = nblocks
+        self.o_parts = torch.empty((nblocks, B, n, H, d), dtype=torch.bfloat16, device=device)
+        self.lse_parts = torch.empty((nblocks, B, H, n), dtype=torch.float32, device=device)
+        self.i = 0
+
+    def block(self, q, k, v, causal):
+        from . import attention_fwd
+        i = self.i
+        self.i += 1
+        return attention_fwd(q, k, v, causal=causal, scale=self.scale, out=self.o_parts[i], lse=self.lse_parts[i])
+
+    def merge(self, o_t, lse_t, first, last):
+        import torch
+        from . import fa_attn_merge
+        if not last:
+            return None
+        if self.nblocks == 1:
+            return self.o_parts[0], self.lse_parts[0]
+        B, n, H, d = self.shape
+        o = torch.empty((B, n, H, d), dtype=torch.bfloat16, device=self.o_parts.device)
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=self.o_parts.device)
+        fa_attn_merge(self.o_parts, self.lse_parts, self.nblocks, o, lse, B, n, H, d)
+        return o, lse
+
+
+def _gpu_rank(q, rank, world, causal, scale):
+    nblocks = sum(mode != "skip" for _, _, mode in ring_schedule(rank, world, causal))
+    return _GpuRank(tuple(q.shape), nblocks, scale, q.device)
+
+
+def ring_attention_fwd(q, k, v, causal=True, scale=None, group=None):
+    """Sequence-parallel exact attention over the ranks of `group`.
+
+    q [B, n, Hq, d], k, v [B, n, Hkv, d] bf16 on this rank's GPU: this rank's
+    shard (tokens rank*n .. rank*n + n - 1) of sequences of length n*R.
+    Returns (o [B, n, Hq, d] bf16, lse [B, Hq, n] fp32) for this rank's query
+    rows, over all keys of the sequence."""
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    d = q.shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    g = _gpu_rank(q, r, R, causal, scale)
+    return ring_forward(q, ring_exchange(k, v, group), r, R, causal, g.block, g.merge)
+
+
+def ring_attention_fwd_local(q_shards, k_shards, v_shards, causal=True, scale=None):
+    """The ring of R ranks run by one process on one GPU: shard r of each
+    list plays rank r, and hop t of rank r reads shard (r - t) mod R straight
+    from the lists instead of receiving it. Same blocks, kernels and merge
+    order as `ring_attention_fwd`; for checking and timing the per-rank work
+    where only one GPU is at hand. Returns per-rank (o, lse)."""
+    R = len(q_shards)
+    d = q_shards[0].shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    outs = []
+    for r in range(R):
+        blocks = (((r - t) % R, k_shards[(r - t) % R], v_shards[(r - t) % R]) for t in range(R))
+        g = _gpu_rank(q_shards[r], r, R, causal, scale)
+        outs.append(ring_forward(q_shards[r], blocks, r, R, causal, g.block, g.merge))
+    return outs
