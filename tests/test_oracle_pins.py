@@ -339,3 +339,82 @@ def test_kvcache_split_merge_reproduces_whole_cache():
     Om, Lm = oracle.merge_partials(outs, lses)
     np.testing.assert_allclose(Om, O, atol=1e-12)
     np.testing.assert_allclose(Lm.transpose(0, 2, 1), L, atol=1e-12)
+
+
+# ---------------------------------------------------------------- fp8 incoherent processing
+# Pins of oracle/quant.py: Sylvester's Hadamard matrix, the float32 butterfly
+# transform against it, the invariance of the scores under the orthogonal
+# rotation, and the block-scaled e4m3 quantiser (amax -> 448, RNE, zero
+# blocks, ragged last block).
+
+def test_hadamard_definition():
+    H2 = oracle.hadamard(2)
+    assert np.array_equal(H2, np.array([[1.0, 1.0], [1.0, -1.0]]))
+    for d in (1, 4, 64, 128):
+        H = oracle.hadamard(d)
+        assert np.array_equal(H, H.T)
+        assert np.array_equal(np.abs(H), np.ones((d, d)))
+        assert np.array_equal(H @ H.T, d * np.eye(d))
+    with pytest.raises(ValueError):
+        oracle.hadamard(96)
+
+
+def test_fwht_matches_matrix_exactly_on_integers():
+    rng = np.random.default_rng(5)
+    for d in (2, 8, 64, 128):
+        x = rng.integers(-1000, 1000, (7, d)).astype(np.float32)  # every partial sum exact in float32
+        assert np.array_equal(oracle.fwht_f32(x), (x.astype(np.float64) @ oracle.hadamard(d)).astype(np.float32))
+
+
+def test_rotation_spreads_a_one_hot_outlier_evenly():
+    d = 128
+    x = np.zeros((1, d), dtype=np.float32)
+    x[0, 37] = 20.0
+    y = oracle.rotate_f32(x)
+    # row 37 of H has entries +-1: every entry becomes +-20/sqrt(d)
+    assert np.allclose(np.abs(y), 20.0 / np.sqrt(d), rtol=1e-6)
+    assert np.array_equal(np.sign(y[0]), oracle.hadamard(d)[37])
+
+
+def test_rotation_preserves_scores_and_attention():
+    rng = np.random.default_rng(6)
+    B, N, H, d = 1, 40, 2, 64
+    q = rng.standard_normal((B, N, H, d))
+    k = rng.standard_normal((B, N, H, d))
+    v = rng.standard_normal((B, N, H, d))
+    R = oracle.hadamard(d) / np.sqrt(d)  # orthogonal
+    assert np.abs(R @ R.T - np.eye(d)).max() < 1e-14
+    O0, L0 = oracle.attn_fwd(q, k, v, True, 0.125)
+    O1, L1 = oracle.attn_fwd(q @ R, k @ R, v, True, 0.125)
+    assert np.abs(O0 - O1).max() < 1e-12 and np.abs(L0 - L1).max() < 1e-12
+    # the float32 butterfly rotation agrees with the fp64 matrix to float32 accuracy
+    qr = oracle.rotate_f32(q.astype(np.float32))
+    assert np.abs(qr - q @ R).max() < 1e-5
+
+
+def test_quantize_blockscaled_pins():
+    rng = np.random.default_rng(7)
+    B, N, H, d = 2, 300, 2, 64  # three blocks, the last one 44 rows
+    x = rng.standard_normal((B, N, H, d)).astype(np.float32)
+    x[1, 256:, 1] = 0.0  # an all-zero block
+    codes, s = oracle.quantize_blockscaled(x)
+    assert s.shape == (B, H, 3) and s[1, 1, 2] == 1.0
+    assert np.all(codes[1, 256:, 1] == 0)
+    for b in range(B):
+        for h in range(H):
+            for j in range(3):
+                blk = x[b, j * 128:(j + 1) * 128, h]
+                c = codes[b, j * 128:(j + 1) * 128, h]
+                amax = np.abs(blk).max()
+                if amax == 0:
+                    continue
+                assert s[b, h, j] == np.float32(amax) / np.float32(448.0)
+                assert np.abs(c).max() == 448.0  # the block's largest entry maps to the largest code
+                err = np.abs(c.astype(np.float64) * s[b, h, j] - blk)
+                # e4m3: 3 mantissa bits (relative half-step 2^-4), subnormal step 2^-9 (half 2^-10)
+                assert np.all(err <= np.maximum(np.abs(blk) * 2.0 ** -4, s[b, h, j] * 2.0 ** -10) * (1 + 1e-6))
+    # round to nearest even at e4m3 midpoints (spacing 1/8 in [1, 2))
+    y = np.array([448.0, 1.0625, 1.1875, -1.0625], dtype=np.float32).reshape(1, 4, 1, 1)
+    c, s1 = oracle.quantize_blockscaled(y)
+    assert s1[0, 0, 0] == 1.0
+    assert list(c.reshape(-1)) == [448.0, 1.0, 1.25, -1.0]
