@@ -49,9 +49,10 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
-    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring"],
+    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring", "fp8"],
                     help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
-                         "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated)")
+                         "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated); "
+                         "fp8: Hadamard-rotated e4m3 quantisation + fp8 forward (B=2 H=16 N=8192 d=128 causal)")
     ap.add_argument("--ring-shape", default="1,32,8,16384,128",
                     help="B,Hq,Hkv,N,d of the ring workload (causal; N split over the ring)")
     ap.add_argument("--ring-ranks", type=int, default=4, help="ranks emulated on one GPU (--gpus 1)")
@@ -783,8 +784,227 @@ def run_ring_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------- fp8 workload
+
+FP8_METRIC = "fp8 attention forward TFLOP/s (e4m3, Hadamard-rotated Q/K, causal)"
+FP8_SHAPE = (2, 16, 8192, 128)  # B, H, N, d
+
+
+def fp8_inputs(seed=0):
+    """Q, K, V as fp32 with 0.1% of entries x20 (outlier channels), drawn in
+    the order Q, K, V, and their bf16 roundings (what the quantiser reads)."""
+    import numpy as np
+    import synth
+    B, H, N, d = FP8_SHAPE
+    rng = np.random.default_rng(seed)
+    f32 = []
+    for _ in range(3):
+        x = synth.normal_f32(rng, (B, N, H, d))
+        x = np.where(rng.random(size=x.shape) < 1e-3, x * np.float32(20.0), x).astype(np.float32)
+        f32.append(x)
+    return f32, [synth.to_bf16(x) for x in f32]
+
+
+def fp8_sample_rows(N, count=64, seed=2):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(N, size=count - 2, replace=False).tolist()) | {0, N - 1}
+    return np.array(sorted(rows))
+
+
+def run_fp8(args):
+    import numpy as np
+    import torch
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_fp8_reference(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    import oracle
+    B, H, N, d = FP8_SHAPE
+    f32, bf = fp8_inputs(rank)
+    q, k, v = (t.to(dev) for t in bf)
+    scale = 1.0 / math.sqrt(d)
+    nblk = (N + 127) // 128
+    codes = [torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=dev) for _ in range(3)]
+    scl = [torch.empty((B, H, nblk), dtype=torch.float32, device=dev) for _ in range(3)]
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def quantize(rotate_qk=True):
+        for i, (x, rot) in enumerate(((q, rotate_qk), (k, rotate_qk), (v, False))):
+            fa.fa_fp8_quantize(x, codes[i], scl[i], B, N, H, d, int(rot), sptr)
+
+    def forward():
+        fa.fa_fwd_fp8(codes[0], codes[1], codes[2], scl[0], scl[1], scl[2], o, lse, B, H, H, N, d, 1, scale, sptr)
+
+    # error against fp64 attention on the unquantised fp32 values (sampled rows)
+    rows = fp8_sample_rows(N)
+    rows_h = np.tile(rows[None, :], (H, 1))
+    O_ref, _ = oracle.attn_fwd_rows(f32[0][:1], f32[1][:1], f32[2][:1], True, scale, rows_h)
+    errs = {}
+    for rot in (False, True):
+        quantize(rot)
+        forward()
+        torch.cuda.synchronize(dev)
+        got = o[:1].cpu().double().numpy()[:, rows].transpose(0, 2, 1, 3)  # [1,H,R,d]
+        errs["rotated" if rot else "plain"] = oracle.rel_rms(got, O_ref)
+
+    for _ in range(args.warmup):
+        quantize()
+        forward()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            quantize()
+            ev[i][1].record(stream)
+            forward()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    st = fa.fa_get_status(sptr)
+    if st != fa.FA_OK:
+        raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    f_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    tot_ms = (q_ms + f_ms) * args.steps
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    flops = fwd_flops(B, H, N, d, True)
+    value = flops * world * args.steps / (tot_ms * 1e-3) / 1e12
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    ach = flops / (f_ms * 1e-3) / 1e12
+    q_bytes = 3 * B * N * H * d * (2 + 1) + 3 * B * H * nblk * 4
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel (fp8)", "achieved": ach, "peak": fp8_peak,
+                "unit": "TFLOP/s", "frac": ach / fp8_peak, "traffic": None,
+                "peak_source": f"{pk['source']} bf16 burst x 2 (nominal e4m3/bf16 ratio)",
+                "note": "S = Q K^T runs at the e4m3 rate, O += P V at the 16-bit rate (P and V as f16): "
+                        "at most 4/3 of the bf16 peak for this kernel",
+                "quantize_ms": q_ms, "forward_ms": f_ms,
+                "quantize_gbs": q_bytes / (q_ms * 1e-3) / 1e9, "quantize_frac_hbm": q_bytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = [t.pin_memory() for t in bf]
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        l_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for x, hsrc in zip((q, k, v), pin):
+                x.copy_(hsrc, non_blocking=True)
+            quantize()
+            forward()
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * 2 for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4}
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, nr, el, cores = fp8_oracle_sample(args.cpu_budget_s)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{nr} (head, query row) pairs of the workload, fp64 numpy, {el:.1f} s"}
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = {"workload": f"fp8-e4m3 causal forward from bf16 inputs with 0.1% outliers x20, B={B} Hq=Hkv={H} N={N} "
+                       f"d={d}: Q, K rotated by H_d/sqrt(d), per-(head,128-row block) scales",
+           "B": B, "Hq": H, "Hkv": H, "N": N, "d": d, "causal": True,
+           "parallelism": f"dp{world}" if world > 1 else "single", "l2": "flushed before every step",
+           "error_vs_fp64_unquantised": errs, "error_sample": f"{len(rows)} query rows x {H} heads of batch 0"}
+    line = {"metric": FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": 4 * args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def fp8_oracle_sample(budget_s):
+    """The oracle's rotation + quantisation + attention on sampled query rows
+    of one head until `budget_s` is spent: (TFLOP/s, rows, seconds, cores)."""
+    import numpy as np
+    import oracle
+    B, H, N, d = FP8_SHAPE
+    f32, _ = fp8_inputs(0)
+    q, k, v = (x[:1, :, :1] for x in f32)
+    done, el, flops = 0, 0.0, 0.0
+    rng = np.random.default_rng(3)
+    while el < budget_s and done < N:
+        rows = np.sort(rng.choice(N, size=64, replace=False))
+        t0 = time.perf_counter()
+        cq, sq = oracle.quantize_blockscaled(oracle.rotate_f32(q))
+        ck, sk = oracle.quantize_blockscaled(oracle.rotate_f32(k))
+        cv, sv = oracle.quantize_blockscaled(v)
+        oracle.attn_fwd_rows(oracle.dequantize_blockscaled(cq, sq), oracle.dequantize_blockscaled(ck, sk),
+                             oracle.dequantize_blockscaled(cv, sv), True, 1 / math.sqrt(d), rows[None, :])
+        el += time.perf_counter() - t0
+        flops += float(sum(4.0 * (r + 1) * d for r in rows))
+        done += 64
+    return flops / el / 1e12, done, el, os.cpu_count()
+
+
+def run_fp8_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    per = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+    vals = [fp8_oracle_sample(per) for _ in range(args.warmup + args.steps)][args.warmup:]
+    tf = sum(v[0] for v in vals) / len(vals)
+    B, H, N, d = FP8_SHAPE
+    line = {"metric": FP8_METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sum(v[2] for v in vals) / len(vals) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"fp8-e4m3 causal forward, B={B} Hq=Hkv={H} N={N} d={d}, rotated Q/K",
+                       "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+                             "sample": f"{vals[-1][1]} query rows of one head per step, fp64 numpy"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "fp8":
+        return run_fp8(args)
     if args.workload == "ring":
         return run_ring(args)
     if args.workload == "decode":

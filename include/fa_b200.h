@@ -203,6 +203,24 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
 int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d);
 
 /*
+ * Block-scaled e4m3 inputs for fa_fwd_fp8, with optional incoherent
+ * processing (the FA-3 summary's lower-error FP8, contribution 3; the
+ * technique is not named there, this rotation is the reading taken): with
+ * rotate = 1 each row is first multiplied by the orthogonal Hadamard matrix
+ * H_d / sqrt(d) (Sylvester's construction; fast Walsh-Hadamard butterflies in
+ * fp32, stage widths 1, 2, ..., d/2, then one multiply by fp32(1/sqrt(d))).
+ * Rotate Q and K, not V: (Q H)(K H)^T = Q K^T.
+ *   x      DEVICE bf16 [B,N,H,d], 8-byte aligned (in);
+ *   codes  DEVICE e4m3 [B,N,H,d], 4-byte aligned (out);
+ *   scales DEVICE fp32 [B,H,ceil(N/128)] (out): per (batch, head, 128-row
+ *          block) s = amax / 448 in fp32 (1 for an all-zero block); codes are
+ *          the round-to-nearest-even e4m3 of the fp32 quotient (x or x H/sqrt d) / s.
+ *   d = 64 or 128. One kernel on `stream`, bound by HBM.
+ */
+fa_status_t fa_fp8_quantize(const void* x, void* codes, float* scales, int B, int N, int H, int d, int rotate,
+                            void* stream);
+
+/*
  * Merge of attention partials over disjoint key sets (the multi-GPU variants
  * of the topic page "Flash Attention and Efficient Transformer Mechanisms";
  * used by context-parallel ring attention): partial t is exact attention of

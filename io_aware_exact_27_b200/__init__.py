@@ -45,6 +45,7 @@ _SIGS = {
     "fa_set_exp_emulation": [_I],
     "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
     "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
+    "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -139,6 +140,30 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_byt
 def fa_attn_merge(o_parts, lse_parts, nparts, o, lse, B, N, H, d, stream=None):
     _check(_lib.fa_attn_merge(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, N, H, d,
                               _stream(stream)), "fa_attn_merge")
+
+
+def fa_fp8_quantize(x, codes, scales, B, N, H, d, rotate, stream=None):
+    _check(_lib.fa_fp8_quantize(_ptr(x), _ptr(codes), _ptr(scales), B, N, H, d, int(rotate), _stream(stream)),
+           "fa_fp8_quantize")
+
+
+def quantize_fp8(x, rotate=False, stream=None):
+    """x [B,N,H,d] bf16 (CUDA) -> (codes [B,N,H,d] float8_e4m3fn, scales [B,H,ceil(N/128)] f32)."""
+    import torch
+    B, N, H, d = x.shape
+    codes = torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=x.device)
+    scales = torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    fa_fp8_quantize(x, codes, scales, B, N, H, d, rotate, stream)
+    return codes, scales
+
+
+def attention_fwd_fp8_rotated(q, k, v, causal=False, scale=None, stream=None):
+    """bf16 q [B,N,Hq,d], k/v [B,N,Hkv,d] (CUDA) -> (o bf16, lse f32): Q and K
+    rotated by H_d/sqrt(d) and quantised, V quantised, then the fp8 forward."""
+    q8, qs = quantize_fp8(q, True, stream)
+    k8, ks = quantize_fp8(k, True, stream)
+    v8, vs = quantize_fp8(v, False, stream)
+    return attention_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, scale=scale, stream=stream)
 
 
 def fa_fwd_kvcache_workspace_size(B, Nq, Hq, d, num_splits) -> int:

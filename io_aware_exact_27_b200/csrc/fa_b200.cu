@@ -13,6 +13,7 @@
 #include "fa_bwd_kernel.cuh"
 #include "fa_decode_kernel.cuh"
 #include "fa_merge_kernel.cuh"
+#include "fa_quant_kernel.cuh"
 
 namespace {
 
@@ -610,6 +611,34 @@ fa_status_t fa_attn_merge(const void* o_parts, const float* lse_parts, int npart
     fa::fa_merge_kernel<128><<<static_cast<int>(blocks), 256, 0, s>>>(a);
   else
     fa::fa_merge_kernel<64><<<static_cast<int>(blocks), 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status_t fa_fp8_quantize(const void* x, void* codes, float* scales, int B, int N, int H, int d, int rotate,
+                            void* stream) {
+  if (B < 0 || N < 0 || H <= 0 || (rotate != 0 && rotate != 1)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!x || !codes || !scales || !aligned(x, 8) || !aligned(codes, 4) || !aligned(scales, 4))
+    return FA_ERR_INVALID_ARG;
+  const int nblk = (N + 127) / 128;
+  if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;
+  fa::QuantArgs a{};
+  a.x = x;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.B = B;
+  a.N = N;
+  a.H = H;
+  a.nblk = nblk;
+  a.rotate = rotate;
+  a.rscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  dim3 grid(nblk, H, B);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    fa::fa_quant_kernel<128><<<grid, 256, 0, s>>>(a);
+  else
+    fa::fa_quant_kernel<64><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
