@@ -246,3 +246,38 @@ def attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal: bool, scale: fl
                 O[b, i, h] = np.exp(row - lse) @ v[b, :Lb, g]
                 LSE[b, h, i] = lse
     return O, LSE
+
+
+def attn_bwd_block(q, k, v, dout, o, lse, causal: bool, scale: float):
+    """Gradient contributions of one key block when the query rows' softmax
+    statistics come from attention over a larger key set (context-parallel
+    ring attention, reading of the topic page's multi-GPU variants).
+
+    q, dout, o [B,N,Hq,d] and lse [B,Hq,N]: the query rows with the O and LSE
+    of their full attention; k, v [B,Nk,Hkv,d]: one key block (causal: the
+    block on the diagonal, key j hidden from query i when j > i). With
+    P = exp(S - LSE) on this block, D = rowsum(dout * o):
+        dV = P^T dout,  dS = P * (dout V^T - D),  dQ = scale dS K,  dK = scale dS^T q
+    (dK, dV summed over the query heads of a kv head). Summed over disjoint key
+    blocks these give the gradient of the full attention (pinned).
+    Returns (dq, dk, dv) float64."""
+    q, k, v, do, o, L = _f64(q), _f64(k), _f64(v), _f64(dout), _f64(o), _f64(lse)
+    B, N, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            S = scale * (q[b, :, h] @ k[b, :, g].T)
+            if causal:
+                S = np.where(np.arange(Nk)[None, :] > np.arange(N)[:, None], -np.inf, S)
+            P = np.exp(S - L[b, h][:, None])
+            D = (do[b, :, h] * o[b, :, h]).sum(axis=1, keepdims=True)
+            dP = do[b, :, h] @ v[b, :, g].T
+            dS = P * (dP - D)
+            dq[b, :, h] = scale * (dS @ k[b, :, g])
+            dk[b, :, g] += scale * (dS.T @ q[b, :, h])
+            dv[b, :, g] += P.T @ do[b, :, h]
+    return dq, dk, dv

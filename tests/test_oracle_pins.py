@@ -418,3 +418,35 @@ def test_quantize_blockscaled_pins():
     c, s1 = oracle.quantize_blockscaled(y)
     assert s1[0, 0, 0] == 1.0
     assert list(c.reshape(-1)) == [448.0, 1.0, 1.25, -1.0]
+
+
+def test_block_gradients_sum_to_full_gradient():
+    """Ring backward (reading): the per-key-block contributions, each using
+    the full rows' O and LSE, add up to the gradient of full attention; the
+    causal sequence split into R shards: diagonal blocks causal, earlier
+    blocks full, later blocks absent."""
+    rng = np.random.default_rng(9)
+    B, N, Hq, Hkv, d, R = 2, 24, 4, 2, 8, 3
+    q, k, v, do = (rng.standard_normal((B, N, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+    sc = 0.35
+    for causal in (True, False):
+        O, L = oracle.attn_fwd(q, k, v, causal, sc)
+        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, sc)
+        n = N // R
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        for r in range(R):
+            qs = slice(r * n, (r + 1) * n)
+            for src in range(R):
+                if causal and src > r:
+                    continue
+                ks = slice(src * n, (src + 1) * n)
+                a, bb, c = oracle.attn_bwd_block(q[:, qs], k[:, ks], v[:, ks], do[:, qs], O[:, qs], L[:, :, qs],
+                                                 causal and src == r, sc)
+                dq[:, qs] += a
+                dk[:, ks] += bb
+                dv[:, ks] += c
+        assert np.abs(dq - dq_ref).max() < 1e-12
+        assert np.abs(dk - dk_ref).max() < 1e-12
+        assert np.abs(dv - dv_ref).max() < 1e-12
