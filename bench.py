@@ -688,6 +688,41 @@ def run_ring(args):
                 "merge_ms_per_step": m_ms / args.steps,
                 "note": "per-launch flops: a full n x n block 4*B*Hq*n^2*d, the causal diagonal block half of it"}
     clocks = clk.summary()
+    # the ring backward on the same shards (dO drawn after Q, K, V), timed on its own
+    bwd = None
+    if not args.no_bwd:
+        do_h = synth.qkv_bf16(0, B, N, Hq, Hkv, d, with_dout=True)[3]
+        dos = {r: sh(do_h, r).to(dev) for r in range(R)}
+        fw = step()
+        outs = dict(zip(mine, fw))
+
+        def bstep():
+            if world > 1:
+                return [rg.ring_attention_bwd(qs[rank], ks[rank], vs[rank], outs[rank][0], outs[rank][1],
+                                              dos[rank], causal=True, scale=scale)]
+            return rg.ring_attention_bwd_local([qs[r] for r in range(R)], [ks[r] for r in range(R)],
+                                               [vs[r] for r in range(R)], [outs[r][0] for r in range(R)],
+                                               [outs[r][1] for r in range(R)], [dos[r] for r in range(R)],
+                                               causal=True, scale=scale)
+        for _ in range(max(1, args.warmup)):
+            bstep()
+        torch.cuda.synchronize(dev)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            bstep()
+        b1.record(stream)
+        torch.cuda.synchronize(dev)
+        b_ms = b0.elapsed_time(b1)
+        if pg:
+            t = torch.tensor([b_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            b_ms = float(t.item())
+        bwd = {"ms_per_step": b_ms / args.steps,
+               "tflops": 2.5 * f_job * args.steps / (b_ms * 1e-3) / 1e12,
+               "note": "ring backward timed separately: flops 2.5x the forward (five GEMMs)"}
+        if fa.fa_get_status() != fa.FA_OK:
+            raise SystemExit("device status error in the ring backward")
     # end to end: this process's shards copied in from pinned host memory,
     # its O and LSE copied out, every step
     e2e = None
@@ -737,7 +772,7 @@ def run_ring(args):
     line = {"metric": RING_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "backward": bwd,
             "gpu_launches": len(rec) + len(recm)}
     print(json.dumps(line), flush=True)
     return 0

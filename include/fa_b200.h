@@ -239,6 +239,19 @@ fa_status_t fa_attn_merge(const void* o_parts, const float* lse_parts, int npart
 
 
 /*
+ * Sum of gradient partials over key blocks (context-parallel ring attention
+ * backward: the dQ, dK, dV contributions of the key shards):
+ *   acc[i] = (first ? 0 : acc[i]) + part[i];  out[i] = bf16(acc[i]) if out.
+ *   acc  DEVICE fp32 [count], 16-byte aligned (in/out);
+ *   part DEVICE bf16 [count], 16-byte aligned, or NULL (adds nothing);
+ *   out  DEVICE bf16 [count], 16-byte aligned, or NULL.
+ *   count a multiple of 8. One elementwise kernel on `stream`.
+ * The pages have no counterpart; it is the sum in the gradient of a
+ * partitioned key set.
+ */
+fa_status_t fa_grad_accumulate(float* acc, const void* part, void* out, long long count, int first, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (FA_OK if no kernel reported an error since the last
  * call). Returns FA_ERR_CUDA if the synchronisation itself failed.

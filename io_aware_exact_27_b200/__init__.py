@@ -46,6 +46,7 @@ _SIGS = {
     "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
     "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
     "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "fa_grad_accumulate": [_P, _P, _P, ctypes.c_longlong, _I, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -140,6 +141,11 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_byt
 def fa_attn_merge(o_parts, lse_parts, nparts, o, lse, B, N, H, d, stream=None):
     _check(_lib.fa_attn_merge(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, N, H, d,
                               _stream(stream)), "fa_attn_merge")
+
+
+def fa_grad_accumulate(acc, part, out, count, first, stream=None):
+    _check(_lib.fa_grad_accumulate(_ptr(acc), _ptr(part), _ptr(out), int(count), int(first), _stream(stream)),
+           "fa_grad_accumulate")
 
 
 def fa_fp8_quantize(x, codes, scales, B, N, H, d, rotate, stream=None):

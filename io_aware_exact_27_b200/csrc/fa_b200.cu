@@ -642,6 +642,23 @@ fa_status_t fa_fp8_quantize(const void* x, void* codes, float* scales, int B, in
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status_t fa_grad_accumulate(float* acc, const void* part, void* out, long long count, int first, void* stream) {
+  if (count < 0 || count % 8 != 0 || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
+  if (count == 0) return FA_OK;
+  if (!acc || !aligned(acc, 16) || (part && !aligned(part, 16)) || (out && !aligned(out, 16)))
+    return FA_ERR_INVALID_ARG;
+  fa::AccArgs a{};
+  a.acc = acc;
+  a.part = part;
+  a.out = out;
+  a.n8 = count / 8;
+  a.first = first;
+  const long long blocks = (a.n8 + 255) / 256;
+  if (blocks > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  fa::fa_grad_accumulate_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status_t fa_get_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   int w = 0;

@@ -89,4 +89,45 @@ __global__ void __launch_bounds__(256) fa_merge_kernel(const MergeArgs a) {
   }
 }
 
+// Sum of gradient partials over key blocks (ring attention backward): acc
+// (fp32) = part, or acc + part, 8 elements per thread (16-byte bf16 loads);
+// with `out`, also bf16(acc). part may be null (only the conversion).
+struct AccArgs {
+  float* acc;
+  const void* part;  // bf16 or null
+  void* out;         // bf16 or null
+  long long n8;      // count / 8
+  int first;
+};
+
+__global__ void __launch_bounds__(256) fa_grad_accumulate_kernel(const AccArgs a) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= a.n8) return;
+  float4* accp = reinterpret_cast<float4*>(a.acc) + 2 * i;
+  float v[8];
+  if (a.first) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.f;
+  } else {
+    const float4 x0 = accp[0], x1 = accp[1];
+    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+  }
+  if (a.part != nullptr) {
+    const uint4 p = __ldg(reinterpret_cast<const uint4*>(a.part) + i);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&p);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(p2[e]);
+      v[2 * e] += f.x;
+      v[2 * e + 1] += f.y;
+    }
+  }
+  accp[0] = make_float4(v[0], v[1], v[2], v[3]);
+  accp[1] = make_float4(v[4], v[5], v[6], v[7]);
+  if (a.out != nullptr)
+    reinterpret_cast<uint4*>(a.out)[i] =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
 }  // namespace fa

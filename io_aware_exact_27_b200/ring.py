@@ -1,4 +1,4 @@
-"""Context-parallel ring attention (forward) over torch.distributed ranks.
+"""Context-parallel ring attention (forward and backward) over torch.distributed ranks.
 
 The topic page "Flash Attention and Efficient Transformer Mechanisms" (opening
 paragraph) says the method extends to multi-GPU settings for very long
@@ -20,9 +20,15 @@ receive from r-1 into a second buffer). Each block's bf16 (O_t, LSE_t) goes
 to its own slot; after the last block `fa_attn_merge` combines the slots in
 fp32 (one pass over them).
 
-Only the exchange of K/V shards crosses GPUs; the arithmetic of every step runs
-in the library's kernels. The contiguous sharding gives causal ranks unequal
-work (rank r computes r + 1 blocks).
+The backward walks the same ring: each block runs the single-GPU backward
+kernels with the full rows' O and LSE, dQ is summed on the rank, and the fp32
+dK/dV accumulators of a shard travel with it and come home after the last hop
+(see the backward section below).
+
+Only the exchange of K/V shards (and, in the backward, their gradient
+accumulators) crosses GPUs; the arithmetic of every step runs in the
+library's kernels. The contiguous sharding gives causal ranks unequal work
+(rank r computes r + 1 blocks).
 """
 
 from __future__ import annotations
@@ -168,3 +174,169 @@ def ring_attention_fwd_local(q_shards, k_shards, v_shards, causal=True, scale=No
         g = _gpu_rank(q_shards[r], r, R, causal, scale)
         outs.append(ring_forward(q_shards[r], blocks, r, R, causal, g.block, g.merge))
     return outs
+
+
+# ---------------------------------------------------------------- backward
+#
+# With the forward's O and LSE of this rank's query rows (over all keys), the
+# gradient splits over key shards exactly: for the block (my queries, shard
+# src), P = exp(S - LSE), D = rowsum(dO * O), and the block adds
+# dQ += scale dS K_src, dK_src += scale dS^T Q, dV_src += P^T dO with
+# dS = P * (dO V_src^T - D) -- what the single-GPU backward kernels compute
+# when given the full rows' O and LSE. dQ stays on the rank; the fp32 dK/dV
+# accumulators of a shard travel with it and come home after the last hop.
+
+
+def _p2p_exchange(group=None):
+    """send(list) to rank+1 and receive into recv(list) from rank-1, as one
+    batch of point-to-point ops; returns a handle whose wait() completes it."""
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    nxt = dist.get_global_rank(group, (r + 1) % R) if group is not None else (r + 1) % R
+    prv = dist.get_global_rank(group, (r - 1) % R) if group is not None else (r - 1) % R
+
+    class _Handle:
+        def __init__(self, reqs):
+            self.reqs = reqs
+
+        def wait(self):
+            for req in self.reqs:
+                req.wait()
+
+    def exchange(send, recv):
+        ops = [dist.P2POp(dist.isend, t, nxt, group) for t in send]
+        ops += [dist.P2POp(dist.irecv, t, prv, group) for t in recv]
+        return _Handle(dist.batch_isend_irecv(ops))
+
+    return exchange
+
+
+def ring_backward(k, v, rank: int, world: int, causal: bool, block_grad, new_acc, add, exchange):
+    """Transport-agnostic ring backward for one rank.
+
+    block_grad(k, v, causal) -> (dk_t, dv_t): this rank's queries against one
+    key shard (it folds its own dq contribution in); new_acc(x) -> an
+    accumulator shaped like x; add(acc, part, first) sets or adds in place;
+    exchange(send, recv) -> handle (send to rank+1, receive from rank-1).
+    Returns (dk_acc, dv_acc) of this rank's own key shard."""
+    sched = ring_schedule(rank, world, causal)
+    cur = [k, v]
+    acc = [new_acc(k), new_acc(v)]
+    if world > 1:
+        spare = [x.new_empty(x.shape) for x in cur]
+        acc_spare = [new_acc(k), new_acc(v)]
+    for t, src, mode in sched:
+        kv_move = exchange(cur, spare) if t + 1 < world else None  # overlaps the block
+        if mode != "skip":
+            dk_t, dv_t = block_grad(cur[0], cur[1], mode == "causal")
+            add(acc[0], dk_t, t == 0)  # hop 0 is the own shard: always computed
+            add(acc[1], dv_t, t == 0)
+        if world > 1:  # the accumulators follow their shard (home after the last hop)
+            exchange(acc, acc_spare).wait()
+            acc, acc_spare = acc_spare, acc
+        if kv_move is not None:
+            kv_move.wait()
+            cur, spare = spare, cur
+    return acc[0], acc[1]
+
+
+class _GpuRankBwd:
+    """The query side of one rank's backward on the GPU: the D / base-2 LSE
+    workspace prepared once, one fa_bwd_part call per key block, dQ summed in
+    fp32 by fa_grad_accumulate."""
+
+    def __init__(self, q, o, lse, do, Hkv, scale):
+        import torch
+        from . import fa_bwd_workspace_size
+        B, n, Hq, d = q.shape
+        self.q, self.o, self.lse, self.do = q, o, lse, do
+        self.dims = (B, Hq, Hkv, n, d)
+        self.scale = scale
+        self.ws_bytes = fa_bwd_workspace_size(B * n, B, Hq, d)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=q.device)
+        self.dq_t = torch.empty_like(q)
+        self.dk_t = torch.empty((B, n, Hkv, d), dtype=q.dtype, device=q.device)
+        self.dv_t = torch.empty_like(self.dk_t)
+        self.dq_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        self.prepared = False
+        self.first = True
+
+    def block(self, k, v, causal):
+        from . import FA_BWD_DKDV, FA_BWD_DQ, FA_BWD_PREPARE, fa_bwd_part, fa_grad_accumulate
+        B, Hq, Hkv, n, d = self.dims
+        parts = FA_BWD_DKDV | FA_BWD_DQ | (0 if self.prepared else FA_BWD_PREPARE)
+        fa_bwd_part(parts, self.q, k, v, self.o, self.lse, self.do, self.dq_t, self.dk_t, self.dv_t, self.ws,
+                    self.ws_bytes, B, Hq, Hkv, n, d, causal, self.scale)
+        self.prepared = True
+        fa_grad_accumulate(self.dq_acc, self.dq_t, None, self.dq_t.numel(), self.first)
+        self.first = False
+        return self.dk_t, self.dv_t
+
+    def dq(self):
+        import torch
+        from . import fa_grad_accumulate
+        out = torch.empty_like(self.q)
+        fa_grad_accumulate(self.dq_acc, None, out, out.numel(), 0)
+        return out
+
+
+def _gpu_acc_ops():
+    import torch
+    from . import fa_grad_accumulate
+
+    def new_acc(x):
+        return torch.empty(x.shape, dtype=torch.float32, device=x.device)
+
+    def add(acc, part, first):
+        fa_grad_accumulate(acc, part, None, part.numel(), first)
+
+    def to_bf16(acc):
+        out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
+        fa_grad_accumulate(acc, None, out, acc.numel(), 0)
+        return out
+
+    return new_acc, add, to_bf16
+
+
+def ring_attention_bwd(q, k, v, o, lse, do, causal=True, scale=None, group=None):
+    """Gradients of ring attention over the ranks of `group`: this rank's
+    shards q, do, o [B,n,Hq,d], lse [B,Hq,n] (from ring_attention_fwd) and
+    k, v [B,n,Hkv,d] -> (dq, dk, dv) bf16 for this rank's shards."""
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    d = q.shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    g = _GpuRankBwd(q, o, lse, do, k.shape[2], scale)
+    new_acc, add, to_bf16 = _gpu_acc_ops()
+    dk, dv = ring_backward(k, v, r, R, causal, g.block, new_acc, add, _p2p_exchange(group))
+    return g.dq(), to_bf16(dk), to_bf16(dv)
+
+
+def ring_attention_bwd_local(q_shards, k_shards, v_shards, o_shards, lse_shards, do_shards, causal=True,
+                             scale=None):
+    """The ring backward of R ranks run by one process on one GPU, hop by hop
+    (at hop t every rank r works on shard (r - t) mod R, whose accumulators
+    receive their partials in the same hop order as on the ring). For
+    checking where only one GPU is at hand. Returns per-rank (dq, dk, dv)."""
+    R = len(q_shards)
+    d = q_shards[0].shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    new_acc, add, to_bf16 = _gpu_acc_ops()
+    gs = [_GpuRankBwd(q_shards[r], o_shards[r], lse_shards[r], do_shards[r], k_shards[r].shape[2], scale)
+          for r in range(R)]
+    acc_k = [new_acc(x) for x in k_shards]
+    acc_v = [new_acc(x) for x in v_shards]
+    for t in range(R):
+        for r in range(R):
+            src = (r - t) % R
+            mode = ring_block_mode(r, src, causal)
+            if mode == "skip":
+                continue
+            dk_t, dv_t = gs[r].block(k_shards[src], v_shards[src], mode == "causal")
+            add(acc_k[src], dk_t, t == 0)
+            add(acc_v[src], dv_t, t == 0)
+    return [(gs[r].dq(), to_bf16(acc_k[r]), to_bf16(acc_v[r])) for r in range(R)]

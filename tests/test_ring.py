@@ -95,3 +95,59 @@ def test_ring_on_cpu_ranks(world, causal):
     for p in procs:
         p.join(timeout=60)
     assert all(r is None for r in results), results
+
+
+def _rank_bwd_main(rank, world, port, causal, B, N, Hq, Hkv, d, errs):
+    from io_aware_exact_27_b200.ring import _p2p_exchange, ring_backward
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(4)
+        q, k, v, do = (rng.standard_normal((B, N, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+        scale = 1.0 / math.sqrt(d)
+        O, L = oracle.attn_fwd(q, k, v, causal, scale)
+        n = N // world
+        sl = slice(rank * n, (rank + 1) * n)
+        q_r, do_r, o_r, l_r = q[:, sl], do[:, sl], O[:, sl], L[:, :, sl]
+        dq = np.zeros_like(q_r)
+
+        def block_grad(kk, vv, c):
+            a, bb, cc = oracle.attn_bwd_block(q_r, kk.numpy(), vv.numpy(), do_r, o_r, l_r, c, scale)
+            dq[...] += a
+            return torch.from_numpy(bb), torch.from_numpy(cc)
+
+        def add(acc, part, first):
+            if first:
+                acc.copy_(part)
+            else:
+                acc.add_(part)
+
+        k_r = torch.from_numpy(np.ascontiguousarray(k[:, sl]))
+        v_r = torch.from_numpy(np.ascontiguousarray(v[:, sl]))
+        dk, dv = ring_backward(k_r, v_r, rank, world, causal, block_grad, lambda x: torch.zeros_like(x), add,
+                               _p2p_exchange())
+        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, scale)
+        e = max(float(np.abs(dq - dq_ref[:, sl]).max()), float(np.abs(dk.numpy() - dk_ref[:, sl]).max()),
+                float(np.abs(dv.numpy() - dv_ref[:, sl]).max()))
+        errs.put(None if e <= 1e-12 else f"rank {rank}: max |d grad| {e:.3g}")
+    except Exception as e:  # reported to the parent
+        errs.put(f"rank {rank}: {type(e).__name__}: {e}")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (2, False), (3, True)])
+def test_ring_backward_on_cpu_ranks(world, causal):
+    ctx = mp.get_context("spawn")
+    errs = ctx.Queue()
+    port = _free_port()
+    B, N, Hq, Hkv, d = 2, 16 * world, 4, 2, 8
+    procs = [ctx.Process(target=_rank_bwd_main, args=(r, world, port, causal, B, N, Hq, Hkv, d, errs))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [errs.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(r is None for r in results), results
