@@ -281,3 +281,35 @@ def attn_bwd_block(q, k, v, dout, o, lse, causal: bool, scale: float):
             dk[b, :, g] += scale * (dS.T @ q[b, :, h])
             dv[b, :, g] += P.T @ do[b, :, h]
     return dq, dk, dv
+
+
+def attn_fwd_blocksparse(q, k, v, block_mask, causal: bool, scale: float, block: int = 128):
+    """Attention with a block-sparse mask (the topic page's block-sparse
+    variant; its layout is a reading): key j is hidden from query i when
+    block_mask[h, i // block, j // block] == 0 (and, with causal, when j > i).
+    q [B,N,Hq,d]; k, v [B,N,Hkv,d]; block_mask [Hq, ceil(N/block),
+    ceil(N/block)], shared by the batch. A row that sees no key has O = 0 and
+    LSE = -inf. Returns O [B,N,Hq,d], LSE [B,Hq,N] (float64)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    M = np.asarray(block_mask) != 0
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    blk = np.arange(N) // block
+    O = np.zeros((B, N, Hq, v.shape[3]))
+    L = np.full((B, Hq, N), -np.inf)
+    for h in range(Hq):
+        g = kv_head_of(h, Hq, Hkv)
+        visible = M[h][blk[:, None], blk[None, :]]
+        if causal:
+            visible &= np.arange(N)[None, :] <= np.arange(N)[:, None]
+        for b in range(B):
+            S = np.where(visible, scale * (q[b, :, h] @ k[b, :, g].T), -np.inf)
+            rows = visible.any(axis=1)
+            if not rows.any():
+                continue
+            Sr = S[rows]
+            m = Sr.max(axis=1, keepdims=True)
+            lse = m[:, 0] + np.log(np.exp(Sr - m).sum(axis=1))
+            O[b, rows, h] = np.exp(Sr - lse[:, None]) @ v[b, :, g]
+            L[b, h, rows] = lse
+    return O, L

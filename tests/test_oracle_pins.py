@@ -450,3 +450,50 @@ def test_block_gradients_sum_to_full_gradient():
         assert np.abs(dq - dq_ref).max() < 1e-12
         assert np.abs(dk - dk_ref).max() < 1e-12
         assert np.abs(dv - dv_ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------- block-sparse masks
+
+def test_blocksparse_pins():
+    rng = np.random.default_rng(12)
+    B, N, Hq, Hkv, d, blk = 2, 40, 4, 2, 8, 8  # 5 blocks of 8 (small block size: the definition's parameter)
+    q, k, v = (rng.standard_normal((B, N, H, d)) for H in (Hq, Hkv, Hkv))
+    nb = N // blk
+    sc = 0.3
+    ones = np.ones((Hq, nb, nb), dtype=np.uint8)
+    for causal in (False, True):
+        # all blocks on: plain attention
+        O, L = oracle.attn_fwd_blocksparse(q, k, v, ones, causal, sc, blk)
+        O0, L0 = oracle.attn_fwd(q, k, v, causal, sc)
+        assert np.abs(O - O0).max() < 1e-12 and np.abs(L - L0).max() < 1e-12
+    # block lower-triangular mask with causal: the same as causal alone
+    tri = np.tril(ones)
+    O, L = oracle.attn_fwd_blocksparse(q, k, v, tri, True, sc, blk)
+    O0, L0 = oracle.attn_fwd(q, k, v, True, sc)
+    assert np.abs(O - O0).max() < 1e-12
+    # block-diagonal mask: each block attends only itself (= separate sequences)
+    diag = np.broadcast_to(np.eye(nb, dtype=np.uint8), (Hq, nb, nb)).copy()
+    O, L = oracle.attn_fwd_blocksparse(q, k, v, diag, False, sc, blk)
+    cu = np.arange(0, N + 1, blk)
+    for b in range(B):
+        Ov, Lv = oracle.attn_fwd_varlen(q[b], k[b], v[b], cu, False, sc)
+        assert np.abs(O[b] - Ov).max() < 1e-12 and np.abs(L[b] - Lv).max() < 1e-12
+    # a query block with no visible key block: O = 0, LSE = -inf; other rows unaffected
+    m = ones.copy()
+    m[1, 2, :] = 0
+    O, L = oracle.attn_fwd_blocksparse(q, k, v, m, False, sc, blk)
+    assert np.all(O[:, 2 * blk:3 * blk, 1] == 0) and np.all(L[:, 1, 2 * blk:3 * blk] == -np.inf)
+    O0, L0 = oracle.attn_fwd(q, k, v, False, sc)
+    assert np.abs(O[:, :, 0] - O0[:, :, 0]).max() < 1e-12
+    # brute force on one row: a visible-key softmax written out
+    m = (rng.random((Hq, nb, nb)) < 0.5).astype(np.uint8)
+    m[:, :, 0] = 1
+    O, L = oracle.attn_fwd_blocksparse(q, k, v, m, True, sc, blk)
+    b, i, h = 1, 27, 3
+    g = oracle.kv_head_of(h, Hq, Hkv)
+    keys = [j for j in range(N) if j <= i and m[h, i // blk, j // blk]]
+    s = np.array([sc * float(np.dot(q[b, i, h], k[b, j, g])) for j in keys])
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    assert np.abs(O[b, i, h] - sum(pj * v[b, j, g] for pj, j in zip(p, keys))).max() < 1e-12
+    assert abs(L[b, h, i] - (s.max() + np.log(np.exp(s - s.max()).sum()))) < 1e-12
