@@ -203,6 +203,22 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_split
 int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d);
 
 /*
+ * Forward pass with a block-sparse mask (the topic page's block-sparse
+ * variant, which it calls approximate: only the listed blocks are attended;
+ * the mask layout is a reading). As fa_fwd, plus
+ *   block_mask DEVICE uint8 [Hq][nb][nb], nb = ceil(N/128): key block j
+ *              (keys 128j .. 128j+127) is visible to query block i of query
+ *              head h when block_mask[h][i][j] != 0; the same mask for every
+ *              sequence of the batch; with causal = 1 the causal mask applies
+ *              too.
+ * Only visited key blocks are loaded and multiplied. A query row that sees no
+ * key gets O = 0 and LSE = -inf. NULL mask: FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask, void* o,
+                               float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                               void* stream);
+
+/*
  * Block-scaled e4m3 inputs for fa_fwd_fp8, with optional incoherent
  * processing (the FA-3 summary's lower-error FP8, contribution 3; the
  * technique is not named there, this rotation is the reading taken): with

@@ -47,6 +47,7 @@ _SIGS = {
     "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
     "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
     "fa_grad_accumulate": [_P, _P, _P, ctypes.c_longlong, _I, _P],
+    "fa_fwd_blocksparse": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -141,6 +142,22 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_byt
 def fa_attn_merge(o_parts, lse_parts, nparts, o, lse, B, N, H, d, stream=None):
     _check(_lib.fa_attn_merge(_ptr(o_parts), _ptr(lse_parts), int(nparts), _ptr(o), _ptr(lse), B, N, H, d,
                               _stream(stream)), "fa_attn_merge")
+
+
+def fa_fwd_blocksparse(q, k, v, block_mask, o, lse, B, Hq, Hkv, N, d, causal, scale, stream=None):
+    _check(_lib.fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(block_mask), _ptr(o), _ptr(lse), B, Hq, Hkv, N,
+                                   d, int(causal), float(scale), _stream(stream)), "fa_fwd_blocksparse")
+
+
+def attention_fwd_blocksparse(q, k, v, block_mask, causal=False, scale=None, stream=None):
+    """q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16, block_mask uint8 [Hq, ceil(N/128), ceil(N/128)] (CUDA)
+    -> (o [B,N,Hq,d] bf16, lse [B,Hq,N] f32)."""
+    import torch
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    fa_fwd_blocksparse(q, k, v, block_mask, o, lse, B, Hq, k.shape[2], N, d, causal, _default_scale(d, scale), stream)
+    return o, lse
 
 
 def fa_grad_accumulate(acc, part, out, count, first, stream=None):

@@ -35,7 +35,7 @@ struct DeviceState {
   int sms = 0;
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
-  bool fwd_attr[3][6] = {};
+  bool fwd_attr[3][6][2] = {};  // [bf16 d64, bf16 d128, fp8][EMU][block-sparse]
   bool bwd_attr[2] = {false, false};
   bool dec_attr[2] = {false, false};
 };
@@ -108,16 +108,16 @@ fa_status_t check_common(const void* q, const void* k, const void* v, const void
   return FA_OK;
 }
 
-template <int D, int EMU, bool F8 = false>
+template <int D, int EMU, bool F8 = false, bool SPARSE = false>
 fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, fa::FwdArgs a, int tokens,
                        long long units_bound, cudaStream_t stream) {
   constexpr int STAGES = F8 ? 6 : 4;
   using Smem = fa::FwdSmem<D, STAGES, F8>;
-  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU, F8>;
+  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU, F8, SPARSE>;
   const int smem = static_cast<int>(sizeof(Smem)) + 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->fwd_attr[F8 ? 2 : (D == 128 ? 1 : 0)][EMU];
+    bool& done = ds->fwd_attr[F8 ? 2 : (D == 128 ? 1 : 0)][EMU][SPARSE ? 1 : 0];
     if (!done) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -141,7 +141,8 @@ fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void
 }
 
 fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int nseq,
-                         int N, int total_T, int Hq, int Hkv, int d, int causal, float scale, void* stream) {
+                         int N, int total_T, int Hq, int Hkv, int d, int causal, float scale, void* stream,
+                         const uint8_t* block_mask = nullptr) {
   fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
   if (st != FA_OK) return st;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
@@ -159,6 +160,8 @@ fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, f
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.block_mask = block_mask;
+  a.nqb = (N + fa::kBM - 1) / fa::kBM;
   const long long nlev = (N + 255) / 256;
   long long bound;
   if (cu == nullptr) {
@@ -174,6 +177,9 @@ fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, f
   }
   if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (block_mask != nullptr)  // block-sparse: MUFU exponentials only
+    return d == 128 ? launch_fwd<128, 0, false, true>(ds, q, k, v, a, total_T, bound, s)
+                    : launch_fwd<64, 0, false, true>(ds, q, k, v, a, total_T, bound, s);
   switch ((d == 128 ? 10 : 0) + g_exp_emu.load()) {
     case 0: return launch_fwd<64, 0>(ds, q, k, v, a, total_T, bound, s);
     case 2: return launch_fwd<64, 2>(ds, q, k, v, a, total_T, bound, s);
@@ -393,6 +399,15 @@ int dec_chunk_keys(int Ncache, int num_splits) {
 }  // namespace
 
 extern "C" {
+
+fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask, void* o,
+                               float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                               void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return FA_OK;
+  if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  return fwd_dispatch(q, k, v, o, lse, nullptr, B, N, B * N, Hq, Hkv, d, causal, scale, stream, block_mask);
+}
 
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                    int d, int causal, float scale, void* stream) {

@@ -57,6 +57,10 @@ struct FwdArgs {
   uint64_t timeout_ns;
   int* status;
   int inject;      // test hook: 1 = the producer never loads the first K tile
+  // block-sparse: [Hq][nqb][nqb] uint8, key block j visible to query block i
+  // of head h when nonzero (shared by the batch); null = dense
+  const uint8_t* block_mask;
+  int nqb;
   // fp8 only: block scales [B, H, nblk_s] (value = code * scale)
   const float* q_scale;
   const float* k_scale;
@@ -164,6 +168,31 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
 }
 
+// Block-sparse walk over the key blocks [0, jend) of a unit (query blocks
+// qb0, qb0 + 1 of head h): a block is visited when either query block may see
+// it. A unit whose query blocks see no key block still visits block 0, with
+// every score masked (O = 0, LSE = -inf), so that every role runs the same
+// pipeline. Without a mask every block is visited.
+__device__ __forceinline__ bool kv_block_on(const FwdArgs& a, int h, int qb, int j) {
+  return qb < a.nqb && __ldg(a.block_mask + (static_cast<size_t>(h) * a.nqb + qb) * a.nqb + j) != 0;
+}
+__device__ __forceinline__ int next_kv_block(const FwdArgs& a, int h, int qb0, int j, int jend) {
+  if (a.block_mask == nullptr) return j + 1;
+  for (int jj = j + 1; jj < jend; ++jj)
+    if (kv_block_on(a, h, qb0, jj) || kv_block_on(a, h, qb0 + 1, jj)) return jj;
+  return jend;
+}
+__device__ __forceinline__ int first_kv_block(const FwdArgs& a, int h, int qb0, int jend) {
+  const int j = next_kv_block(a, h, qb0, -1, jend);
+  return j < jend ? j : 0;
+}
+__device__ __forceinline__ int count_kv_blocks(const FwdArgs& a, int h, int qb0, int jend) {
+  if (a.block_mask == nullptr) return jend;
+  int n = 0;
+  for (int j = next_kv_block(a, h, qb0, -1, jend); j < jend; j = next_kv_block(a, h, qb0, j, jend)) ++n;
+  return n > 0 ? n : 1;
+}
+
 // Exponentials of 2*NP consecutive columns of one row: p = 2^(s*cj - m),
 // packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[NP] for
 // the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs;
@@ -194,7 +223,7 @@ __device__ __forceinline__ float exp_pack(const float* s, float cj, float m, flo
   return a.x + a.y;
 }
 
-template <int D, int STAGES, int EMU, bool F8>
+template <int D, int STAGES, int EMU, bool F8, bool SPARSE = false>
 __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -267,7 +296,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         const int u = unit_of(rnd, blockIdx.x, gridDim.x);
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
-        const int nblk = num_kv_blocks(un, args.causal);
+        const int jend = num_kv_blocks(un, args.causal);
+        const int nblk = SPARSE ? count_kv_blocks(args, un.h, un.qb2 * 2, jend) : jend;
         const int hkv = un.h / group;
         if (!mbar_wait(smem_u32(&sm.q_empty), (it & 1) ^ 1, abort, args.timeout_ns)) {
           report_error(args.status, kStatusTimeout, 1);
@@ -280,7 +310,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         load_tile<D, EB>(smem_u32(sm.q[0]), &tm_q, qbar, un.h, row0);
         load_tile<D, EB>(smem_u32(sm.q[1]), &tm_q, qbar, un.h, row0 + kBM);
         q_issued = it + 1;
-        for (int j = 0; j < nblk && ok; ++j) {
+        int jb = SPARSE ? first_kv_block(args, un.h, un.qb2 * 2, jend) : 0;  // key block of the j-th visit
+        for (int j = 0; j < nblk && ok; ++j, jb = SPARSE ? next_kv_block(args, un.h, un.qb2 * 2, jb, jend) : jb + 1) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_prod % STAGES;
             if (!mbar_wait(smem_u32(&sm.kv_empty[slot]), ((kv_prod / STAGES) & 1) ^ 1, abort, args.timeout_ns)) {
@@ -293,7 +324,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
             } else {
               const uint32_t bar = smem_u32(&sm.kv_full[slot]);
               mbar_expect_tx(bar, Smem::kTileBytes);
-              load_tile<D, EB>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
+              load_tile<D, EB>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + jb * kBN);
             }
             ++kv_prod;
           }
@@ -320,7 +351,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         const int u = unit_of(rnd, blockIdx.x, gridDim.x);
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
-        const int nblk = num_kv_blocks(un, args.causal);
+        const int nblk =
+            SPARSE ? count_kv_blocks(args, un.h, un.qb2 * 2, num_kv_blocks(un, args.causal)) : num_kv_blocks(un, args.causal);
         if (!(ok = wait(&sm.q_full, it & 1, 10))) break;
         const uint32_t q0 = smem_u32(sm.q[0]), q1 = smem_u32(sm.q[1]);
         uint32_t slotK = kv_cons % STAGES;
@@ -389,7 +421,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         const int u = unit_of(rnd, blockIdx.x, gridDim.x);
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
-        const int nblk = num_kv_blocks(un, args.causal);
+        const int nblk =
+            SPARSE ? count_kv_blocks(args, un.h, un.qb2 * 2, num_kv_blocks(un, args.causal)) : num_kv_blocks(un, args.causal);
         for (int j = 0; j < nblk; ++j, ++g) {
           const uint32_t idx = 2 * g + 1;  // ring index of V_j (K and V alternate)
           const uint32_t slot = idx % STAGES;
@@ -450,7 +483,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       const int u = unit_of(rnd, blockIdx.x, gridDim.x);
       if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
-      const int nblk = num_kv_blocks(un, args.causal);
+      const int jend = num_kv_blocks(un, args.causal);
+      const int nblk = SPARSE ? count_kv_blocks(args, un.h, un.qb2 * 2, jend) : jend;  // key blocks visited
       const int row = un.qb2 * 2 * kBM + tile * kBM + r_in_tile;  // row within the sequence
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;  // last visible key
       // scores are kept in base-2 units t = s * cj; cj = scale*log2(e) for
@@ -462,15 +496,16 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         if (qt < args.nblk_s) sq = args.q_scale[(static_cast<size_t>(un.seq) * args.Hq + un.h) * args.nblk_s + qt];
         kvs = (static_cast<size_t>(un.seq) * args.Hkv + un.h / group) * args.nblk_s;
         sv_max = 0.f;
-        for (int jj = 0; jj < nblk; ++jj) sv_max = fmaxf(sv_max, args.v_scale[kvs + jj]);
+        for (int jj = 0; jj < jend; ++jj) sv_max = fmaxf(sv_max, args.v_scale[kvs + jj]);
         sv_max = fmaxf(sv_max, 1e-30f);
       }
       float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
-      for (int j = 0; j < nblk; ++j) {
+      int jb = SPARSE ? first_kv_block(args, un.h, un.qb2 * 2, jend) : 0;  // key block of the j-th visit
+      for (int j = 0; j < nblk; ++j, jb = SPARSE ? next_kv_block(args, un.h, un.qb2 * 2, jb, jend) : jb + 1) {
         float cj = cl, pmul = 1.f;
         if constexpr (F8) {
-          cj = cl * sq * args.k_scale[kvs + j];
-          pmul = args.v_scale[kvs + j] / sv_max;
+          cj = cl * sq * args.k_scale[kvs + jb];
+          pmul = args.v_scale[kvs + jb] / sv_max;
         }
         // every lane waits; the outcome is made warp-uniform so that the
         // warp-collective tcgen05 loads below run converged
@@ -481,9 +516,11 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         }
         ++sc;
         tc_fence_after();
-        const int kv0 = j * kBN + 64 * half;  // first key of this half
+        const int kv0 = jb * kBN + 64 * half;  // first key of this half
+        // block-sparse: the whole block is hidden from this tile (uniform over the tile)
+        const bool tile_on = !SPARSE || kv_block_on(args, un.h, un.qb2 * 2 + tile, jb);
         // warp-uniform: every lane of a warp takes the same masked/unmasked path
-        const bool masked_blk = __any_sync(0xffffffffu, kv0 + 63 > limit);
+        const bool masked_blk = !tile_on || __any_sync(0xffffffffu, kv0 + 63 > limit);
         // pass 1: this half's row maximum, exchanged with the partner half
         float pm;
         {
@@ -493,7 +530,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
           if (masked_blk) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
-              if (kv0 + c > limit) sv[c] = -INFINITY;
+              if (!tile_on || kv0 + c > limit) sv[c] = -INFINITY;
           }
           float a = fmax3(sv[0], sv[1], sv[2]);
           float b = fmax3(sv[32], sv[33], sv[34]);
@@ -537,10 +574,12 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
           if (masked_blk) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (kv0 + 32 * c + e > limit) sv[e] = -INFINITY;
+              if (!tile_on || kv0 + 32 * c + e > limit) sv[e] = -INFINITY;
           }
           uint32_t pk[16];
-          lsum += masked_blk ? exp_pack<0, F8, 16>(sv, cj, m_new, pmul, pk)
+          // a row that has seen no visible key yet (block-sparse) keeps
+          // m = -inf: its exponentials are taken against 0 and are all 0
+          lsum += masked_blk ? exp_pack<0, F8, 16>(sv, cj, SPARSE && m_new == -INFINITY ? 0.f : m_new, pmul, pk)
                              : exp_pack<EMU, F8, 16>(sv, cj, m_new, pmul, pk);
           tmem_st16(S + 16 * c, pk);
         }
@@ -568,7 +607,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       const float lt = l + lo;
       const bool valid = row < un.n;
       // fp8: P entered the PV MMA scaled by sv_j / sv_max
-      const float inv_l = (F8 ? sv_max : 1.f) / lt;
+      const float inv_l = !SPARSE || lt > 0.f ? (F8 ? sv_max : 1.f) / lt : 0.f;  // no visible key: O = 0
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
                             (static_cast<size_t>(un.tok0 + row) * args.Hq + un.h) * D + HC * half;
 #pragma unroll 1
@@ -591,7 +630,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       if (valid && half == 0) {
         const size_t li = varlen ? (static_cast<size_t>(un.h) * args.lse_head_stride + un.tok0 + row)
                                  : (static_cast<size_t>(un.seq * args.Hq + un.h) * args.lse_head_stride + row);
-        args.lse[li] = m * 0.6931471805599453f + logf(lt);
+        args.lse[li] = !SPARSE || lt > 0.f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
       }
     }
     if (!ok) sm.abort = 1;
