@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
-    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring", "fp8"],
+    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring", "fp8", "blocksparse"],
                     help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
                          "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated); "
                          "fp8: Hadamard-rotated e4m3 quantisation + fp8 forward (B=2 H=16 N=8192 d=128 causal)")
@@ -1036,8 +1036,207 @@ def run_fp8_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------- block-sparse workload
+
+BS_METRIC = "block-sparse attention forward TFLOP/s over the visible query-key pairs (bf16, causal)"
+BS_SHAPE = (1, 32, 8, 16384, 128)  # B, Hq, Hkv, N, d
+BS_WINDOW = 8  # key blocks of the sliding window (the query's own block and the 7 before it)
+
+
+def bs_mask(Hq, nb):
+    """Sliding window of BS_WINDOW blocks plus block 0 (a global first block), every head."""
+    import numpy as np
+    m = np.zeros((Hq, nb, nb), dtype=np.uint8)
+    for i in range(nb):
+        m[:, i, max(0, i - BS_WINDOW + 1):i + 1] = 1
+        m[:, i, 0] = 1
+    return m
+
+
+def bs_pairs(mask, N, causal=True):
+    """Visible (query, key) pairs of one head under the block mask (and causal)."""
+    import numpy as np
+    nb = mask.shape[1]
+    pairs = 0
+    for i in range(nb):
+        for j in range(nb):
+            if not mask[0, i, j]:
+                continue
+            qi = np.arange(i * 128, min(N, (i + 1) * 128))
+            kj = np.arange(j * 128, min(N, (j + 1) * 128))
+            pairs += int((kj[None, :] <= qi[:, None]).sum()) if causal else qi.size * kj.size
+    return pairs
+
+
+def run_blocksparse(args):
+    import numpy as np
+    import torch
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_bs_reference(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    import synth
+    B, Hq, Hkv, N, d = BS_SHAPE
+    nb = (N + 127) // 128
+    mask_h = bs_mask(Hq, nb)
+    pairs = bs_pairs(mask_h, N)
+    flops = 4.0 * d * pairs * Hq * B
+    q_h, k_h, v_h = synth.qkv_bf16(rank, B, N, Hq, Hkv, d)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    mask = torch.from_numpy(mask_h).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(d)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.fa_fwd_blocksparse(q, k, v, mask, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+
+    def dense():
+        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
+
+    def timed(fn, steps):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    for _ in range(args.warmup):
+        step()
+        dense()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        tot_ms = timed(step, args.steps)
+    dense_ms = timed(dense, args.steps) / args.steps
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    ms = tot_ms / args.steps
+    value = flops * world / (ms * 1e-3) / 1e12
+    pk = peaks()
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel (block-sparse)", "achieved": value / world,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": value / world / pk["bf16_tflops"],
+                "traffic": None, "peak_source": f"{pk['source']} bf16 burst (cuBLAS)",
+                "note": "flops of the visible (query, key) pairs, 4*d each",
+                "dense_causal_ms": dense_ms, "speedup_vs_dense_causal": dense_ms / ms,
+                "pair_density_vs_causal": pairs / (N * (N + 1) / 2)}
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h)]
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        l_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for x, hsrc in zip((q, k, v), pin):
+                x.copy_(hsrc, non_blocking=True)
+            step()
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        e2e = {"value": flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": sum(x.numel() * 2 for x in pin),
+               "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4}
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, nr, el, cores = bs_oracle_sample(args.cpu_budget_s)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{nr} query rows of head 0, fp64 numpy, {el:.1f} s"}
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = {"workload": f"bf16 causal block-sparse forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}: every query "
+                       f"block sees its own and the {BS_WINDOW - 1} previous key blocks plus block 0",
+           "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "parallelism": f"dp{world}" if world > 1 else "single",
+           "l2": "flushed before every step"}
+    line = {"metric": BS_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bs_oracle_sample(budget_s):
+    """The oracle's block-masked attention on sampled query rows of head 0."""
+    import numpy as np
+    import oracle
+    import synth
+    B, Hq, Hkv, N, d = BS_SHAPE
+    q, k, v = synth.qkv_bf16(0, 1, N, 1, 1, d)
+    q, k, v = (t.double().numpy() for t in (q, k, v))
+    nb = (N + 127) // 128
+    m = bs_mask(1, nb)[0]
+    rng = np.random.default_rng(5)
+    done, el, flops = 0, 0.0, 0.0
+    blk = np.arange(N) // 128
+    while el < budget_s and done < N:
+        rows = rng.choice(N, size=32, replace=False)
+        t0 = time.perf_counter()
+        for i in rows:
+            keys = np.nonzero((m[blk[i]][blk] != 0) & (np.arange(N) <= i))[0]
+            s = (q[0, i, 0] @ k[0, keys, 0].T) / math.sqrt(d)
+            p = np.exp(s - s.max())
+            _ = (p / p.sum()) @ v[0, keys, 0]
+            flops += 4.0 * d * keys.size
+        el += time.perf_counter() - t0
+        done += 32
+    return flops / el / 1e12, done, el, os.cpu_count()
+
+
+def run_bs_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return 0
+    per = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+    vals = [bs_oracle_sample(per) for _ in range(args.warmup + args.steps)][args.warmup:]
+    tf = sum(v[0] for v in vals) / len(vals)
+    B, Hq, Hkv, N, d = BS_SHAPE
+    line = {"metric": BS_METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sum(v[2] for v in vals) / len(vals) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"bf16 causal block-sparse forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}",
+                       "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+                             "sample": f"{vals[-1][1]} query rows of head 0 per step, fp64 numpy"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload == "blocksparse":
+        return run_blocksparse(args)
     if args.workload == "fp8":
         return run_fp8(args)
     if args.workload == "ring":
