@@ -7,6 +7,9 @@ pass (dQ, dK, dV) on the workload B=4, Hq=Hkv=16, N=2048, d=128 (Q, K, V, dO
 i.i.d. N(0,1) rounded to bf16, seed 0). Flops: forward 4*B*Hq*N^2*d halved for
 causal, backward 2.5x the forward (five GEMMs instead of two).
 
+The step is timed through the public calls (fa_fwd, fa_bwd); a second pass
+times the kernels one by one for the roofline of the dominant one.
+
 Prints ONE JSON line (rank 0). `--impl reference` times the fp64 CPU oracle
 instead, on a bounded sample of the same workload. Multi-GPU (torchrun):
 every rank runs its own independent batch (weak scaling, no data-path
@@ -263,35 +266,44 @@ def run_ours(args):
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error during warm-up")
 
-    # timed region: K steps, L2 flushed before each (outside the step's events).
-    # The backward runs as its three parts back to back (exactly fa_bwd's
-    # work) with events between them, for the per-kernel roofline.
-    nev = 5 if with_bwd else 2
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    # timed region: K steps through the public calls (fa_fwd, then fa_bwd,
+    # which runs its dQ kernel beside the dK/dV kernel), L2 flushed before
+    # each step (outside the step's events)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
-            e = ev[i]
-            e[0].record(stream)
-            fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
-            e[1].record(stream)
-            if with_bwd:
-                for j, part in enumerate((fa.FA_BWD_PREPARE, fa.FA_BWD_DKDV, fa.FA_BWD_DQ)):
-                    fa.fa_bwd_part(part, q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d,
-                                   int(causal), scale, sptr)
-                    e[2 + j].record(stream)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     st = fa.fa_get_status(sptr)
     if st != fa.FA_OK:
         raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
-    step_ms = [e[0].elapsed_time(e[-1]) for e in ev]
-    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(nev - 1)]
-    tot_ms = sum(step_ms)
+    tot_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    # per-kernel times for the roofline: a second pass with the backward as its
+    # three parts one after another (exactly fa_bwd's work), events between them
+    nev = 5 if with_bwd else 2
+    nseg = max(3, args.steps // 4)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(nseg)]
+    for i in range(nseg):
+        flush.zero_()
+        e = ev2[i]
+        e[0].record(stream)
+        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
+        e[1].record(stream)
+        if with_bwd:
+            for j, part in enumerate((fa.FA_BWD_PREPARE, fa.FA_BWD_DKDV, fa.FA_BWD_DQ)):
+                fa.fa_bwd_part(part, q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d,
+                               int(causal), scale, sptr)
+                e[2 + j].record(stream)
+    torch.cuda.synchronize(dev)
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev2] for j in range(nev - 1)]
     if pg:
         t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)

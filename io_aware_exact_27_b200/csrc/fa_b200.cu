@@ -38,6 +38,10 @@ struct DeviceState {
   bool fwd_attr[3][6][2] = {};  // [bf16 d64, bf16 d128, fp8][EMU][block-sparse]
   bool bwd_attr[2] = {false, false};
   bool dec_attr[2] = {false, false};
+  // the backward runs its dQ kernel beside the dK/dV kernel: a second stream
+  // and two events, created on first use
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -237,17 +241,39 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
     fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
+  fa::BwdArgs akv = a;
+  akv.num_units = static_cast<int>(units_dkdv);
+  const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
+  fa::BwdArgs aq = a;
+  aq.num_units = static_cast<int>(units_dq);
+  const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
+  if ((parts & FA_BWD_DKDV) && (parts & FA_BWD_DQ) && g1 > 0 && g2 > 0) {
+    // dK/dV on the caller's stream and dQ on the side stream, both after the
+    // preparation: their persistent CTAs have uneven causal work, and dQ's
+    // CTAs take the SMs that dK/dV's leave early. The caller's stream waits
+    // for both. Each output is still written by one CTA (deterministic).
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (ds->side == nullptr) {
+      if (cudaStreamCreateWithFlags(&ds->side, cudaStreamNonBlocking) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ds->fork, cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ds->join, cudaEventDisableTiming) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    if (cudaEventRecord(ds->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ds->side, ds->fork, 0) != cudaSuccess)
+      return FA_ERR_CUDA;
+    kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    kdq<<<g2, fa::kThreadsBwd, smem_dq, ds->side>>>(tq, tk, tv, tdo, aq);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaEventRecord(ds->join, ds->side) != cudaSuccess || cudaStreamWaitEvent(stream, ds->join, 0) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
   if (parts & FA_BWD_DKDV) {
-    fa::BwdArgs akv = a;
-    akv.num_units = static_cast<int>(units_dkdv);
-    const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
     if (g1 > 0) kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (parts & FA_BWD_DQ) {
-    fa::BwdArgs aq = a;
-    aq.num_units = static_cast<int>(units_dq);
-    const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
     if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
