@@ -38,6 +38,7 @@ from .attention import (  # noqa: F401
     attn_bwd_block,
     attn_fwd_kvcache,
     attn_fwd_blocksparse,
+    attn_bwd_blocksparse,
     merge_partials,
     dequantize_blockscaled,
 )

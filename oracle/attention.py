@@ -313,3 +313,39 @@ def attn_fwd_blocksparse(q, k, v, block_mask, causal: bool, scale: float, block:
             O[b, rows, h] = np.exp(Sr - lse[:, None]) @ v[b, :, g]
             L[b, h, rows] = lse
     return O, L
+
+
+def attn_bwd_blocksparse(q, k, v, dout, block_mask, causal: bool, scale: float, block: int = 128):
+    """Gradients of sum(O * dout) for attn_fwd_blocksparse (the same mask
+    reading): the analytic gradient of the definition with hidden entries'
+    P = 0; a row that sees no key contributes nothing. Returns dq, dk, dv
+    (float64; dk, dv summed over the query heads of a kv head)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    M = np.asarray(block_mask) != 0
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    blk = np.arange(N) // block
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for h in range(Hq):
+        g = kv_head_of(h, Hq, Hkv)
+        visible = M[h][blk[:, None], blk[None, :]]
+        if causal:
+            visible &= np.arange(N)[None, :] <= np.arange(N)[:, None]
+        rows = visible.any(axis=1)
+        for b in range(B):
+            S = np.where(visible, scale * (q[b, :, h] @ k[b, :, g].T), -np.inf)
+            P = np.zeros_like(S)
+            Sr = S[rows]
+            m = Sr.max(axis=1, keepdims=True)
+            E = np.exp(Sr - m)
+            P[rows] = E / E.sum(axis=1, keepdims=True)
+            O = P @ v[b, :, g]
+            dv[b, :, g] += P.T @ do[b, :, h]
+            dP = do[b, :, h] @ v[b, :, g].T
+            D = (do[b, :, h] * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dq[b, :, h] = scale * (dS @ k[b, :, g])
+            dk[b, :, g] += scale * (dS.T @ q[b, :, h])
+    return dq, dk, dv

@@ -497,3 +497,42 @@ def test_blocksparse_pins():
     p /= p.sum()
     assert np.abs(O[b, i, h] - sum(pj * v[b, j, g] for pj, j in zip(p, keys))).max() < 1e-12
     assert abs(L[b, h, i] - (s.max() + np.log(np.exp(s - s.max()).sum()))) < 1e-12
+
+
+def test_blocksparse_backward_pins():
+    rng = np.random.default_rng(13)
+    B, N, Hq, Hkv, d, blk = 1, 24, 2, 1, 4, 6  # 4 blocks of 6
+    q, k, v, do = (rng.standard_normal((B, N, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+    nb = N // blk
+    sc = 0.4
+    ones = np.ones((Hq, nb, nb), dtype=np.uint8)
+    for causal in (False, True):
+        g = oracle.attn_bwd_blocksparse(q, k, v, do, ones, causal, sc, blk)
+        g0 = oracle.attn_bwd(q, k, v, do, causal, sc)
+        for a, b in zip(g, g0):
+            assert np.abs(a - b).max() < 1e-12
+    # block-diagonal mask: the gradient of separate sequences
+    diag = np.broadcast_to(np.eye(nb, dtype=np.uint8), (Hq, nb, nb)).copy()
+    g = oracle.attn_bwd_blocksparse(q, k, v, do, diag, True, sc, blk)
+    gv = oracle.attn_bwd_varlen(q[0], k[0], v[0], do[0], np.arange(0, N + 1, blk), True, sc)
+    for a, b in zip(g, gv):
+        assert np.abs(a[0] - b).max() < 1e-12
+    # central finite differences of sum(O * dO) on a random mask with an empty query block
+    m = (rng.random((Hq, nb, nb)) < 0.6).astype(np.uint8)
+    m[0, 1, :] = 0
+    dq, dk, dv = oracle.attn_bwd_blocksparse(q, k, v, do, m, True, sc, blk)
+
+    def f(qq, kk, vv):
+        O, _ = oracle.attn_fwd_blocksparse(qq, kk, vv, m, True, sc, blk)
+        return float((O * do).sum())
+
+    eps = 1e-6
+    for arr, grad, idx in ((q, dq, (0, 9, 1, 2)), (k, dk, (0, 3, 0, 1)), (v, dv, (0, 14, 0, 3))):
+        a1, a2 = arr.copy(), arr.copy()
+        a1[idx] += eps
+        a2[idx] -= eps
+        args1 = [a1 if arr is x else x for x in (q, k, v)]
+        args2 = [a2 if arr is x else x for x in (q, k, v)]
+        fd = (f(*args1) - f(*args2)) / (2 * eps)
+        assert abs(fd - grad[idx]) < 1e-6
+    assert np.all(dq[0, 6:12, 0] == 0)  # the empty query block has no gradient
