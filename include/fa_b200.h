@@ -219,6 +219,22 @@ fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, cons
                                void* stream);
 
 /*
+ * Backward pass of fa_fwd_blocksparse: the gradient of the same block-masked
+ * attention (the backward of the topic page's backward-pass section with P
+ * recomputed only on visible blocks; entries of hidden blocks are exactly 0,
+ * so they add nothing to dQ, dK or dV). Arguments as fa_bwd, plus block_mask
+ * exactly as given to fa_fwd_blocksparse (DEVICE uint8 [Hq][nb][nb]); o and
+ * lse are that call's outputs (a row with lse = -inf gets dQ = 0). dQ units
+ * visit only the key blocks their query tile sees; dK/dV units only the
+ * (query head, query tile) steps that see their key tile; a tile that sees
+ * nothing writes zeros. Deterministic. NULL mask: FA_ERR_INVALID_ARG.
+ */
+fa_status_t fa_bwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask,
+                               const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
+                               float scale, void* stream);
+
+/*
  * Block-scaled e4m3 inputs for fa_fwd_fp8, with optional incoherent
  * processing (the FA-3 summary's lower-error FP8, contribution 3; the
  * technique is not named there, this rotation is the reading taken): with

@@ -48,6 +48,7 @@ _SIGS = {
     "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
     "fa_grad_accumulate": [_P, _P, _P, ctypes.c_longlong, _I, _P],
     "fa_fwd_blocksparse": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_bwd_blocksparse": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
@@ -158,6 +159,27 @@ def attention_fwd_blocksparse(q, k, v, block_mask, causal=False, scale=None, str
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     fa_fwd_blocksparse(q, k, v, block_mask, o, lse, B, Hq, k.shape[2], N, d, causal, _default_scale(d, scale), stream)
     return o, lse
+
+
+def fa_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N, d, causal,
+                       scale, stream=None):
+    _check(_lib.fa_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(block_mask), _ptr(o), _ptr(lse), _ptr(dout),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d,
+                                   int(causal), float(scale), _stream(stream)), "fa_bwd_blocksparse")
+
+
+def attention_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, causal=False, scale=None, workspace=None,
+                              stream=None):
+    """Gradients (dq, dk, dv) of sum(o * dout) for attention_fwd_blocksparse with the same block_mask."""
+    import torch
+    B, N, Hq, d = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B * N, B, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    fa_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), B, Hq,
+                       k.shape[2], N, d, causal, _default_scale(d, scale), stream)
+    return dq, dk, dv
 
 
 def fa_grad_accumulate(acc, part, out, count, first, stream=None):

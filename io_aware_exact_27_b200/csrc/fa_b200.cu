@@ -36,7 +36,7 @@ struct DeviceState {
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
   bool fwd_attr[3][6][2] = {};  // [bf16 d64, bf16 d128, fp8][EMU][block-sparse]
-  bool bwd_attr[2] = {false, false};
+  bool bwd_attr[2][2] = {{false, false}, {false, false}};  // [d == 128][block-sparse]
   bool dec_attr[2] = {false, false};
   // the backward runs its dQ kernel beside the dK/dV kernel: a second stream
   // and two events, created on first use
@@ -204,17 +204,17 @@ size_t vec_bytes(int tokens, int nseq, int Hq) {
   return (b + 255) & ~size_t(255);
 }
 
-template <int D>
+template <int D, bool SPARSE = false>
 fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* dout,
                        fa::BwdArgs a, long long units_dq, long long units_dkdv, int parts, cudaStream_t stream) {
   constexpr int STAGES = 4;
-  auto kdq = fa::fa_bwd_dq_kernel<D, STAGES>;
-  auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES>;
+  auto kdq = fa::fa_bwd_dq_kernel<D, STAGES, SPARSE>;
+  auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES, SPARSE>;
   const int smem_dq = static_cast<int>(sizeof(fa::DqSmem<D, STAGES>)) + 1024;
   const int smem_dkv = static_cast<int>(sizeof(fa::DkvSmem<D, STAGES>)) + 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->bwd_attr[D == 128 ? 1 : 0];
+    bool& done = ds->bwd_attr[D == 128 ? 1 : 0][SPARSE ? 1 : 0];
     if (!done) {
       if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess ||
           cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv) != cudaSuccess)
@@ -283,7 +283,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
 fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                          const int* cu, int nseq, int N, int total_T, int Hq, int Hkv, int d, int causal,
-                         float scale, void* stream, int parts = FA_BWD_ALL) {
+                         float scale, void* stream, int parts = FA_BWD_ALL, const uint8_t* block_mask = nullptr) {
   fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
   if (st != FA_OK) return st;
   if (!dout || !dq || !dk || !dv || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
@@ -330,6 +330,11 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   if (udq > INT32_MAX) return FA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (parts <= 0 || parts > FA_BWD_ALL) return FA_ERR_INVALID_ARG;
+  a.block_mask = block_mask;
+  a.nqb = static_cast<int>(nt);
+  if (block_mask != nullptr)
+    return d == 128 ? launch_bwd<128, true>(ds, q, k, v, dout, a, udq, ukv, parts, s)
+                    : launch_bwd<64, true>(ds, q, k, v, dout, a, udq, ukv, parts, s);
   return d == 128 ? launch_bwd<128>(ds, q, k, v, dout, a, udq, ukv, parts, s)
                   : launch_bwd<64>(ds, q, k, v, dout, a, udq, ukv, parts, s);
 }
@@ -515,6 +520,18 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
   if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
   return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
                       causal, scale, stream, parts);
+}
+
+fa_status_t fa_bwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask,
+                               const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
+                               float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
+                      causal, scale, stream, FA_BWD_ALL, block_mask);
 }
 
 fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -52,6 +52,9 @@ struct BwdArgs {
   int num_units;
   uint64_t timeout_ns;
   int* status;
+  // block-sparse: [Hq][nqb][nqb] uint8 as for the forward; null = dense
+  const uint8_t* block_mask;
+  int nqb;
 };
 
 // ------------------------------------------------------------------ pre
@@ -62,6 +65,50 @@ struct BwdArgs {
 // per head hold +inf (LSE) and 0 (D), harmless when a tile runs past the end
 // of its sequence.
 __device__ __forceinline__ int ws_offset(int tok0, int seq) { return ((tok0 + 3) & ~3) + 4 * seq; }
+
+// Block-sparse backward (the forward's mask): key block kb visible to query
+// block qb of query head hq. A dQ unit (query tile qt of head h) walks the key
+// blocks it sees; a dK/dV unit (key tile kb of kv head hk) walks the (query
+// head of the group, query tile) steps that see it. A unit that sees none
+// still runs one block / step, every score masked (zero gradient), so that
+// every role runs the same pipeline.
+__device__ __forceinline__ bool bwd_block_on(const BwdArgs& a, int hq, int qb, int kb) {
+  return __ldg(a.block_mask + (static_cast<size_t>(hq) * a.nqb + qb) * a.nqb + kb) != 0;
+}
+__device__ __forceinline__ int dq_next_block(const BwdArgs& a, int h, int qt, int j, int jend) {
+  for (int jj = j + 1; jj < jend; ++jj)
+    if (bwd_block_on(a, h, qt, jj)) return jj;
+  return jend;
+}
+__device__ __forceinline__ int dq_first_block(const BwdArgs& a, int h, int qt, int jend) {
+  const int j = dq_next_block(a, h, qt, -1, jend);
+  return j < jend ? j : 0;
+}
+__device__ __forceinline__ int dq_count_blocks(const BwdArgs& a, int h, int qt, int jend) {
+  int n = 0;
+  for (int j = dq_next_block(a, h, qt, -1, jend); j < jend; j = dq_next_block(a, h, qt, j, jend)) ++n;
+  return n > 0 ? n : 1;
+}
+// dK/dV step st of a unit: query head hk*group + st / nqt, query tile i0 + st % nqt
+__device__ __forceinline__ int kv_next_step(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb, int st,
+                                            int nsteps) {
+  for (int s2 = st + 1; s2 < nsteps; ++s2)
+    if (bwd_block_on(a, hk * group + s2 / nqt, i0 + s2 % nqt, kb)) return s2;
+  return nsteps;
+}
+__device__ __forceinline__ int kv_first_step(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb,
+                                             int nsteps) {
+  const int s2 = kv_next_step(a, hk, group, nqt, i0, kb, -1, nsteps);
+  return s2 < nsteps ? s2 : 0;
+}
+__device__ __forceinline__ int kv_count_steps(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb,
+                                              int nsteps) {
+  int n = 0;
+  for (int s2 = kv_next_step(a, hk, group, nqt, i0, kb, -1, nsteps); s2 < nsteps;
+       s2 = kv_next_step(a, hk, group, nqt, i0, kb, s2, nsteps))
+    ++n;
+  return n > 0 ? n : 1;
+}
 
 // Workspace entry r = (head h, index i) -> the token it holds, or -1 for a
 // gap / trailing filler entry: the last sequence whose block starts at or
@@ -114,7 +161,11 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdArgs a) {
           gv[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dout) + off));
           const size_t li = a.cu_seqlens ? static_cast<size_t>(h) * a.lse_head_stride + tok[u]
                                          : (static_cast<size_t>(seq) * a.Hq + h) * a.lse_head_stride + row;
-          if (sl == 0) lv[u] = __ldg(a.lse + li);
+          if (sl == 0) {
+            // a row that saw no key (block-sparse: LSE = -inf) gets +inf, so P = 0
+            const float l = __ldg(a.lse + li);
+            lv[u] = l == -INFINITY ? INFINITY : l;
+          }
         }
       }
     }
@@ -179,7 +230,7 @@ __device__ __forceinline__ void issue_ss_nt(uint32_t d_tmem, uint32_t a_smem, ui
   issue_qk<DD>(d_tmem, a_smem, b_smem);
 }
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -241,7 +292,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int u = unit_of(rnd, blockIdx.x, gridDim.x);
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
-        const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
         const int hkv = un.h / group;
         if (!mbar_wait(smem_u32(&sm.q_empty), (it & 1) ^ 1, abort, args.timeout_ns)) {
           report_error(args.status, kStatusTimeout, 30);
@@ -254,7 +306,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         load_tile<D>(smem_u32(sm.q), &tm_q, qbar, un.h, row0);
         load_tile<D>(smem_u32(sm.dout), &tm_do, qbar, un.h, row0);
         q_issued = it + 1;
-        for (int j = 0; j < nblk && ok; ++j) {
+        int jb = SPARSE ? dq_first_block(args, un.h, un.qb2, jend) : 0;  // key block of the j-th visit
+        for (int j = 0; j < nblk && ok; ++j, jb = SPARSE ? dq_next_block(args, un.h, un.qb2, jb, jend) : jb + 1) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_prod % STAGES;
             if (!mbar_wait(smem_u32(&sm.kv_empty[slot]), ((kv_prod / STAGES) & 1) ^ 1, abort, args.timeout_ns)) {
@@ -264,7 +317,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             }
             const uint32_t bar = smem_u32(&sm.kv_full[slot]);
             mbar_expect_tx(bar, Smem::kTileBytes);
-            load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + j * kBN);
+            load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + jb * kBN);
             ++kv_prod;
           }
         }
@@ -289,7 +342,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const int u = unit_of(rnd, blockIdx.x, gridDim.x);
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
-        const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+        const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
         if (!(ok = wait(&sm.q_full, it & 1, 40))) break;
         const uint32_t qa = smem_u32(sm.q), doa = smem_u32(sm.dout);
         // prologue: S(0)
@@ -343,14 +397,16 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const int u = unit_of(rnd, blockIdx.x, gridDim.x);
       if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
-      const int nblk = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+      const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
+      const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
+      int jb = SPARSE ? dq_first_block(args, un.h, un.qb2, jend) : 0;  // key block of the j-th visit
       const int row = un.qb2 * kBM + r_in_tile;
       const bool valid = row < un.n;
       const size_t wi = static_cast<size_t>(un.h) * args.ws_stride + ws_offset(un.tok0, un.seq) + row;
       const float lse2 = valid ? args.lse2[wi] : INFINITY;
       const float dval = valid ? args.dvec[wi] : 0.f;
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;
-      for (int j = 0; j < nblk; ++j) {
+      for (int j = 0; j < nblk; ++j, jb = SPARSE ? dq_next_block(args, un.h, un.qb2, jb, jend) : jb + 1) {
         const int sb = j & 1;
         const uint32_t par = sb ? (sc1 & 1) : (sc0 & 1);
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[sb]), par, abort, args.timeout_ns));
@@ -363,12 +419,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         uint32_t sr[64];
         tmem_ld64(tS0 + sb * 128 + half * 64 + lane_bits, sr);
         float p[64];
-        const int c0 = j * kBN + half * 64;
-        const bool masked_blk = __any_sync(0xffffffffu, c0 + 63 > limit);
+        const int c0 = jb * kBN + half * 64;
+        // block-sparse: a visit of a block this tile may not see (a unit that sees none)
+        const bool off = SPARSE && !bwd_block_on(args, un.h, un.qb2, jb);
+        const bool masked_blk = off || __any_sync(0xffffffffu, c0 + 63 > limit);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -lse2));
-          p[c] = (masked_blk && c0 + c > limit) ? 0.f : x;
+          p[c] = (masked_blk && (off || c0 + c > limit)) ? 0.f : x;
         }
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dp_full), dpc & 1, abort, args.timeout_ns));
         if (!ok) {
@@ -458,7 +516,7 @@ struct DkvSmem {
   int level_count[1024];
 };
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -515,11 +573,19 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   uint32_t prod_issued = 0, kv_issued = 0;
 
   // steps of a unit: (query head of the group, query tile) pairs
+  // (block-sparse: only the steps whose (query tile, key tile) block is on
+  // are visited, at least one per unit so that dK and dV are written)
   auto unit_steps = [&](const Unit& un, int& i0, int& nqt) {
     const int nq = (un.n + 127) / 128;
     i0 = args.causal ? un.qb2 : 0;
     nqt = nq - i0;
     return group * nqt;
+  };
+  auto first_step = [&](const Unit& un, int i0, int nqt, int nsteps) {
+    return SPARSE ? kv_first_step(args, un.h, group, nqt, i0, un.qb2, nsteps) : 0;
+  };
+  auto next_step = [&](const Unit& un, int i0, int nqt, int st, int nsteps) {
+    return SPARSE ? kv_next_step(args, un.h, group, nqt, i0, un.qb2, st, nsteps) : st + 1;
   };
 
   if (warp == 8) {
@@ -531,6 +597,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const Unit un = decode_unit(sched, u);
       int i0, nqt;
       const int nsteps = unit_steps(un, i0, nqt);
+      const int nvis = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nsteps) : nsteps;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.kv_empty), (it & 1) ^ 1, abort, args.timeout_ns));
       if (!ok) {
         if (lane == 0) report_error(args.status, kStatusTimeout, 60);
@@ -543,7 +610,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         load_tile<D>(smem_u32(sm.v), &tm_v, bar, un.h, un.tok0 + un.qb2 * kBN);
       }
       kv_issued = it + 1;
-      for (int st = 0; st < nsteps && ok; ++st) {
+      int st = first_step(un, i0, nqt, nsteps);
+      for (int v = 0; v < nvis && ok; ++v, st = next_step(un, i0, nqt, st, nsteps)) {
         const int hq = un.h * group + st / nqt;
         const int qi = i0 + st % nqt;
         for (int w = 0; w < 2; ++w) {
@@ -591,7 +659,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
         int i0, nqt;
-        const int nsteps = unit_steps(un, i0, nqt);
+        const int nall = unit_steps(un, i0, nqt);
+        const int nsteps = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nall) : nall;  // visited
         if (!(ok = wait(&sm.kv_full, it & 1, 70))) break;
         const uint32_t ka = smem_u32(sm.k), va = smem_u32(sm.v);
         // prologue: S^T(0), dP^T(0)
@@ -660,10 +729,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const Unit un = decode_unit(sched, u);
       int i0, nqt;
       const int nsteps = unit_steps(un, i0, nqt);
+      const int nvis = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nsteps) : nsteps;
       const int key = un.qb2 * kBN + r_in_tile;  // key row within the sequence
       const bool valid = key < un.n;
-      for (int st = 0; st < nsteps; ++st, ++vstep) {
+      int st = first_step(un, i0, nqt, nsteps);
+      for (int v = 0; v < nvis; ++v, ++vstep, st = next_step(un, i0, nqt, st, nsteps)) {
         const int qi = i0 + st % nqt;
+        // block-sparse: the forced visit of a unit that no query tile sees
+        const bool off = SPARSE && !bwd_block_on(args, un.h * group + st / nqt, qi, un.qb2);
         const float* vec = sm.vec[vstep % (STAGES / 2)][0];
         const int q0 = qi * kBM + half * 64;  // first query column of this half
         // the producer stored this step's LSE2/D before arriving on the Q
@@ -685,12 +758,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         tmem_ld64(tS + half * 64 + lane_bits, sr);
         // a query column q is hidden from key k when q >= n or (causal and k > q)
         const int lo = args.causal ? key : 0;  // smallest visible query
-        const bool masked_blk = __any_sync(0xffffffffu, q0 < lo || q0 + 63 >= un.n);
+        const bool masked_blk = off || __any_sync(0xffffffffu, q0 < lo || q0 + 63 >= un.n);
         float p[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -vec[half * 64 + c]));
-          p[c] = (masked_blk && (q0 + c < lo || q0 + c >= un.n)) ? 0.f : x;
+          p[c] = (masked_blk && (off || q0 + c < lo || q0 + c >= un.n)) ? 0.f : x;
         }
         {
           uint32_t pk[32];
