@@ -1119,6 +1119,26 @@ def run_blocksparse(args):
     def dense():
         fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, 1, scale, sptr)
 
+    # the training step's backward over the same mask, timed apart (and the
+    # dense causal backward beside it); flops 2.5x the forward's (five GEMMs)
+    do = synth.qkv_bf16(rank + 100, B, N, Hq, Hkv, d, with_dout=True)[3].to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    o_bs = torch.empty_like(q)
+    lse_bs = torch.empty_like(lse)
+    o_dn = torch.empty_like(q)
+    lse_dn = torch.empty_like(lse)
+    fa.fa_fwd_blocksparse(q, k, v, mask, o_bs, lse_bs, B, Hq, Hkv, N, d, 1, scale, sptr)
+    fa.fa_fwd(q, k, v, o_dn, lse_dn, B, Hq, Hkv, N, d, 1, scale, sptr)
+
+    def bwd_step():
+        fa.fa_bwd_blocksparse(q, k, v, mask, o_bs, lse_bs, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale,
+                              sptr)
+
+    def bwd_dense():
+        fa.fa_bwd(q, k, v, o_dn, lse_dn, do, dq, dk, dv, ws, ws_bytes, B, Hq, Hkv, N, d, 1, scale, sptr)
+
     def timed(fn, steps):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         for e0, e1 in evs:
@@ -1132,6 +1152,8 @@ def run_blocksparse(args):
     for _ in range(args.warmup):
         step()
         dense()
+        bwd_step()
+        bwd_dense()
     torch.cuda.synchronize(dev)
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error during warm-up")
@@ -1141,6 +1163,11 @@ def run_blocksparse(args):
     with ClockSampler(local) as clk:
         tot_ms = timed(step, args.steps)
     dense_ms = timed(dense, args.steps) / args.steps
+    b_ms = timed(bwd_step, args.steps) / args.steps
+    bd_ms = timed(bwd_dense, args.steps) / args.steps
+    bwd = {"ms": b_ms, "tflops": 2.5 * flops / (b_ms * 1e-3) / 1e12, "dense_causal_ms": bd_ms,
+           "speedup_vs_dense_causal": bd_ms / b_ms,
+           "note": "fa_bwd_blocksparse (pre + dK/dV + dQ) on the same mask, per GPU; flops 2.5x the forward's"}
     if pg:
         t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -1192,7 +1219,7 @@ def run_blocksparse(args):
     line = {"metric": BS_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
-            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": args.steps}
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": args.steps, "backward": bwd}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -12,7 +12,8 @@
 // Design (one persistent CTA per SM, 576 threads; 640 for fp8):
 //   warps 0-7   softmax of query tile 0: warp w takes TMEM lanes (rows)
 //               32*(w%4).. and key columns 64*((w/4)%2)..; the two warps of
-//               a row quadrant exchange row maxima and sums through smem
+//               a row quadrant exchange row maxima and sums through smem at
+//               a named barrier of their own
 //   warps 8-15  softmax of query tile 1, likewise
 //   warp  16    TMA producer: Q tiles once per unit, K_j / V_j through a ring
 //   warp  17    tcgen05 issuer (one thread) and TMEM owner
@@ -39,6 +40,9 @@ constexpr int kWarpConv = 18;
 constexpr int kThreadsFwd = 18 * 32;
 constexpr int kThreadsFwdF8 = 20 * 32;
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, base-2 exponent units
+// Named barrier of the two softmax warps that share a query tile's TMEM lane
+// quadrant (ids 1..8; 0 is __syncthreads)
+__host__ __device__ constexpr int fwd_pair_barrier(int tile, int quad) { return 1 + tile * 4 + quad; }
 
 
 struct FwdArgs {
@@ -80,7 +84,6 @@ struct FwdSmem {
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
   uint64_t v16_full[2], v16_empty[2];
-  uint64_t pair_bar[2][4];        // per (tile, lane quadrant): the two column halves
   float xch[2][2][2][128];        // [slot][tile][half][row] values exchanged by a pair
   uint64_t drain;
   uint32_t tmem_base;
@@ -248,7 +251,6 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       mbar_init(smem_u32(&sm.p_full[i]), 8);  // one arrival per softmax warp of the tile
       mbar_init(smem_u32(&sm.o_final[i]), 1);
       mbar_init(smem_u32(&sm.o_free[i]), 8);
-      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&sm.pair_bar[i][q]), 2);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.v16_full[i]), 2);  // one arrival per converter warp
@@ -461,23 +463,24 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     const uint32_t S = tmem + tile * 128 + 64 * half + lane_bits;          // this half of S
     constexpr int HC = D / 2;                                              // O columns per half
     const uint32_t O = tmem + 256 + tile * 128 + HC * half + lane_bits;    // this half of O
-    const uint32_t pair = smem_u32(&sm.pair_bar[tile][quad]);
+    const int pair_bar = fwd_pair_barrier(tile, quad);
     const float cl = args.scale_log2;
     constexpr float tau = kTau;
     uint32_t sc = 0, xc = 0, it = 0;
     bool ok = true;
     // Hands v to the partner warp (same rows, other column half) and returns
-    // its value; two smem slots alternate so a fast warp never overwrites a
-    // value its partner has not read yet. Bounded wait; false on give-up.
-    auto exchange = [&](float v, float& other) -> bool {
+    // its value: a barrier over the pair's 64 threads that also ORs their
+    // failure flags, so both warps leave together and neither waits at the
+    // barrier for a partner that has gone. Two smem slots alternate: a warp
+    // writes slot s again only after the partner has passed the barrier that
+    // follows its read of slot s.
+    auto exchange = [&](bool good, float v, float& other) -> bool {
       const int slot = xc & 1;
-      sm.xch[slot][tile][half][r_in_tile] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pair);
-      const bool w = __all_sync(0xffffffffu, mbar_wait(pair, xc & 1, abort, args.timeout_ns));
+      if (good) sm.xch[slot][tile][half][r_in_tile] = v;
+      const bool fail = bar_red_or(!good, pair_bar, 64);
       ++xc;
       other = sm.xch[slot][tile][half ^ 1][r_in_tile];
-      return w;
+      return !fail;
     };
     for (int rnd = 0; ok; ++rnd, ++it) {
       const int u = unit_of(rnd, blockIdx.x, gridDim.x);
@@ -508,25 +511,23 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
           pmul = args.v_scale[kvs + jb] / sv_max;
         }
         // every lane waits; the outcome is made warp-uniform so that the
-        // warp-collective tcgen05 loads below run converged
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[tile]), sc & 1, abort, args.timeout_ns));
-        if (!ok) {
-          if (lane == 0) report_error(args.status, kStatusTimeout, 20 + tile);
-          break;
-        }
+        // warp-collective tcgen05 loads below run converged, and is shared
+        // with the partner warp at the exchange
+        const bool good =
+            __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[tile]), sc & 1, abort, args.timeout_ns));
         ++sc;
-        tc_fence_after();
         const int kv0 = jb * kBN + 64 * half;  // first key of this half
         // block-sparse: the whole block is hidden from this tile (uniform over the tile)
         const bool tile_on = !SPARSE || kv_block_on(args, un.h, un.qb2 * 2 + tile, jb);
         // warp-uniform: every lane of a warp takes the same masked/unmasked path
         const bool masked_blk = !tile_on || __any_sync(0xffffffffu, kv0 + 63 > limit);
         // pass 1: this half's row maximum, exchanged with the partner half
-        float pm;
-        {
+        float pm = -INFINITY;
+        if (good) {
           uint32_t sr[64];
-          tmem_ld64(S, sr);
           float* sv = reinterpret_cast<float*>(sr);
+          tc_fence_after();
+          tmem_ld64(S, sr);
           if (masked_blk) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -542,9 +543,9 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
           pm = fmax3(fmaxf(a, sv[31]), b, sv[63]);
         }
         float po;
-        if (!exchange(pm, po)) {
+        if (!exchange(good, pm, po)) {
           ok = false;
-          if (lane == 0) report_error(args.status, kStatusTimeout, 24);
+          if (!good && lane == 0) report_error(args.status, kStatusTimeout, 20 + tile);
           break;
         }
         const float mt = fmaxf(pm, po) * cj;  // identical in both halves
@@ -592,18 +593,15 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 (this half's columns), LSE
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[tile]), it & 1, abort, args.timeout_ns));
-      if (!ok) {
-        if (lane == 0) report_error(args.status, kStatusTimeout, 22 + tile);
+      const bool good =
+          __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.o_final[tile]), it & 1, abort, args.timeout_ns));
+      float lo;
+      if (!exchange(good, l, lo)) {
+        ok = false;
+        if (!good && lane == 0) report_error(args.status, kStatusTimeout, 22 + tile);
         break;
       }
       tc_fence_after();
-      float lo;
-      if (!exchange(l, lo)) {
-        ok = false;
-        if (lane == 0) report_error(args.status, kStatusTimeout, 26);
-        break;
-      }
       const float lt = l + lo;
       const bool valid = row < un.n;
       // fp8: P entered the PV MMA scaled by sv_j / sv_max
