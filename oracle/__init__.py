@@ -43,5 +43,5 @@ from .attention import (  # noqa: F401
     dequantize_blockscaled,
 )
 from .tiled import attn_head_tiled  # noqa: F401
-from .quant import hadamard, fwht_f32, rotate_f32, quantize_blockscaled  # noqa: F401
+from .quant import hadamard, fwht_f32, rotate_f32, quantize_blockscaled, dequantize_f32  # noqa: F401
 from .metrics import max_abs, rel_rms  # noqa: F401

@@ -81,3 +81,22 @@ def quantize_blockscaled(x, block: int = 128):
         q = (xb / s[:, None, :, None]).astype(np.float32)
         codes[:, rows] = torch.from_numpy(np.ascontiguousarray(q)).to(torch.float8_e4m3fn).float().numpy()
     return codes, scales
+
+
+def dequantize_f32(codes, scales, unrotate: bool = False, block: int = 128) -> np.ndarray:
+    """float32 counterpart of attention.dequantize_blockscaled, step by step:
+    the values the fp8 forward attends over, restated in the original space
+    (the input of the fp8 backward, which differentiates attention on them:
+    the straight-through reading of "an fp8 backward").
+    codes float32 [B,N,H,d] holding e4m3 values, scales float32 [B,H,nblk].
+    Steps, each one float32 operation: y = code * s of the row's block; with
+    `unrotate`, the inverse of the rotation, which is the rotation itself
+    (H_d / sqrt(d) is symmetric and orthogonal): the same butterflies as
+    rotate_f32, then the multiply by float32(1/sqrt(d)). Returns float32."""
+    codes = np.asarray(codes, dtype=np.float32)
+    scales = np.asarray(scales, dtype=np.float32)
+    B, N, H, d = codes.shape
+    blk = np.arange(N) // block
+    s = scales[:, :, blk]  # [B, H, N]
+    y = (codes * np.transpose(s, (0, 2, 1))[..., None]).astype(np.float32)
+    return rotate_f32(y) if unrotate else y

@@ -288,6 +288,43 @@ def test_fp8_synth_roundtrip_error_bounded():
     assert np.all(rel[~small] <= 2 ** -4 + 1e-7)
 
 
+def test_dequantize_f32_without_rotation_by_hand():
+    """Power-of-two scales make every product exact: the float32 steps equal
+    the values by hand (and the fp64 definition)."""
+    codes = np.zeros((1, 130, 1, 4), dtype=np.float32)
+    codes[0, 0, 0] = [1.0, -2.0, 448.0, 0.001953125]
+    codes[0, 129, 0] = [3.0, 0.5, -0.75, 0.0]
+    scales = np.array([[[0.25, 4.0]]], dtype=np.float32)
+    x = oracle.dequantize_f32(codes, scales)
+    assert x.dtype == np.float32
+    np.testing.assert_array_equal(x[0, 0, 0], [0.25, -0.5, 112.0, 0.00048828125])
+    np.testing.assert_array_equal(x[0, 129, 0], [12.0, 2.0, -3.0, 0.0])
+    np.testing.assert_array_equal(x, oracle.dequantize_blockscaled(codes, scales))
+
+
+def test_dequantize_f32_unrotate_inverts_the_rotation():
+    """H_d/sqrt(d) is its own inverse (H_d H_d = d I): with unit scales the
+    unrotated values are the codes times H_d / sqrt(d) (closed form, fp64),
+    and quantise(rotate(x)) -> dequantise(unrotate) returns x within the
+    e4m3 step of the rotated block."""
+    rng = np.random.default_rng(3)
+    d = 64
+    codes = torch.from_numpy(rng.standard_normal((1, 5, 2, d)).astype(np.float32)).to(torch.float8_e4m3fn).float()
+    x = oracle.dequantize_f32(codes.numpy(), np.ones((1, 2, 1), dtype=np.float32), unrotate=True)
+    want = codes.double().numpy() @ (oracle.hadamard(d) / np.sqrt(d))
+    np.testing.assert_allclose(x, want, rtol=0, atol=2e-5 * np.abs(want).max())
+    xs = rng.standard_normal((1, 200, 2, d)).astype(np.float32)
+    c, s = oracle.quantize_blockscaled(oracle.rotate_f32(xs))
+    back = oracle.dequantize_f32(c, s, unrotate=True)
+    # each rotated entry is off by at most half an e4m3 step (2**-4 relative,
+    # amax/448 * 2**-9 absolute below the normal range); the orthogonal
+    # unrotation keeps the per-row 2-norm of that error
+    err = np.linalg.norm((back - xs).astype(np.float64), axis=-1)
+    bound = np.linalg.norm(oracle.rotate_f32(xs).astype(np.float64), axis=-1) * 2 ** -4 + \
+        np.sqrt(d) * s.max() * 2 ** -9 + 1e-6
+    assert np.all(err <= bound)
+
+
 # --- decode against a KV cache (bottom-right causal alignment) -------------
 
 def test_kvcache_full_cache_equals_causal_self_attention():
