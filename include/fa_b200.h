@@ -253,6 +253,24 @@ fa_status_t fa_fp8_quantize(const void* x, void* codes, float* scales, int B, in
                             void* stream);
 
 /*
+ * The inverse of fa_fp8_quantize, input of the fp8 backward: bf16 values in
+ * the original space from block-scaled e4m3 codes. The fp8 forward attends
+ * over code * scale (Q, K rotated when quantised with rotate = 1); its
+ * gradient (straight-through reading: the pages describe an fp8 forward
+ * only) is the bf16 backward (fa_bwd, with the fp8 forward's O and LSE) on
+ * these values, with the rotation undone for Q and K, which keeps Q K^T.
+ *   codes  DEVICE e4m3 [B,N,H,d], 4-byte aligned (in);
+ *   scales DEVICE fp32 [B,H,ceil(N/128)] (in), as fa_fp8_quantize writes them;
+ *   x      DEVICE bf16 [B,N,H,d], 8-byte aligned (out): per element, in fp32,
+ *          code * scale; with unrotate = 1 then the butterflies of the fast
+ *          Walsh-Hadamard transform and a multiply by fp32(1/sqrt(d))
+ *          (H_d / sqrt(d) is its own inverse); rounded to nearest even bf16.
+ *   d = 64 or 128. One kernel on `stream`, bound by HBM.
+ */
+fa_status_t fa_fp8_dequantize(const void* codes, const float* scales, void* x, int B, int N, int H, int d,
+                              int unrotate, void* stream);
+
+/*
  * Merge of attention partials over disjoint key sets (the multi-GPU variants
  * of the topic page "Flash Attention and Efficient Transformer Mechanisms";
  * used by context-parallel ring attention): partial t is exact attention of

@@ -46,6 +46,7 @@ _SIGS = {
     "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
     "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
     "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
+    "fa_fp8_dequantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
     "fa_grad_accumulate": [_P, _P, _P, ctypes.c_longlong, _I, _P],
     "fa_fwd_blocksparse": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_blocksparse": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
@@ -200,6 +201,33 @@ def quantize_fp8(x, rotate=False, stream=None):
     scales = torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
     fa_fp8_quantize(x, codes, scales, B, N, H, d, rotate, stream)
     return codes, scales
+
+
+def fa_fp8_dequantize(codes, scales, x, B, N, H, d, unrotate, stream=None):
+    _check(_lib.fa_fp8_dequantize(_ptr(codes), _ptr(scales), _ptr(x), B, N, H, d, int(unrotate), _stream(stream)),
+           "fa_fp8_dequantize")
+
+
+def dequantize_fp8(codes, scales, unrotate=False, stream=None):
+    """codes [B,N,H,d] float8_e4m3fn + scales [B,H,ceil(N/128)] f32 (CUDA) -> bf16 [B,N,H,d]
+    values in the original space (rotation undone with unrotate=True)."""
+    import torch
+    B, N, H, d = codes.shape
+    x = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=codes.device)
+    fa_fp8_dequantize(codes, scales, x, B, N, H, d, unrotate, stream)
+    return x
+
+
+def attention_bwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, dout, causal=False, scale=None, rotated=False,
+                      workspace=None, stream=None):
+    """Gradients (dq, dk, dv) bf16 of sum(o * dout) for the fp8 forward (o, lse from
+    attention_fwd_fp8 on these codes), with respect to the original-space inputs:
+    the codes are dequantised (Q and K unrotated when they were quantised with the
+    rotation) and the bf16 backward runs on them with the fp8 forward's o and lse."""
+    q = dequantize_fp8(q8, q_scale, rotated, stream)
+    k = dequantize_fp8(k8, k_scale, rotated, stream)
+    v = dequantize_fp8(v8, v_scale, False, stream)
+    return attention_bwd(q, k, v, o, lse, dout, causal=causal, scale=scale, workspace=workspace, stream=stream)
 
 
 def attention_fwd_fp8_rotated(q, k, v, causal=False, scale=None, stream=None):

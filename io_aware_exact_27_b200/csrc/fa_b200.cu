@@ -700,6 +700,34 @@ fa_status_t fa_fp8_quantize(const void* x, void* codes, float* scales, int B, in
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status_t fa_fp8_dequantize(const void* codes, const float* scales, void* x, int B, int N, int H, int d,
+                              int unrotate, void* stream) {
+  if (B < 0 || N < 0 || H <= 0 || (unrotate != 0 && unrotate != 1)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!x || !codes || !scales || !aligned(x, 8) || !aligned(codes, 4) || !aligned(scales, 4))
+    return FA_ERR_INVALID_ARG;
+  const int nblk = (N + 127) / 128;
+  if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;
+  fa::DequantArgs a{};
+  a.codes = static_cast<const uint8_t*>(codes);
+  a.scales = scales;
+  a.x = x;
+  a.B = B;
+  a.N = N;
+  a.H = H;
+  a.nblk = nblk;
+  a.unrotate = unrotate;
+  a.rscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  dim3 grid(nblk, H, B);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    fa::fa_dequant_kernel<128><<<grid, 256, 0, s>>>(a);
+  else
+    fa::fa_dequant_kernel<64><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status_t fa_grad_accumulate(float* acc, const void* part, void* out, long long count, int first, void* stream) {
   if (count < 0 || count % 8 != 0 || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
   if (count == 0) return FA_OK;

@@ -125,4 +125,78 @@ __global__ void __launch_bounds__(256) fa_quant_kernel(const QuantArgs a) {
   }
 }
 
+// The inverse map, input of the fp8 backward: bf16 values in the original
+// space from the codes and scales. One CTA per (batch, head, 128-row block),
+// 8 warps x 16 rows; per element, each step one IEEE fp32 operation in a
+// fixed order: code (exact e4m3 -> f16 -> f32) times the block's scale; with
+// `unrotate` the same butterflies and 1/sqrt(D) multiply as the quantiser
+// (H_D / sqrt(D) is its own inverse); round to nearest even bf16.
+struct DequantArgs {
+  const uint8_t* codes;  // [B, N, H, D] e4m3
+  const float* scales;   // [B, H, nblk]
+  void* x;               // [B, N, H, D] bf16 (out)
+  int B, N, H, nblk;
+  int unrotate;
+  float rscale;          // fp32(1/sqrt(D))
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_dequant_kernel(const DequantArgs a) {
+  constexpr int E = D / 32;  // elements per lane
+  constexpr int RPW = 16;    // rows per warp
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const float s = a.scales[(static_cast<size_t>(b) * a.H + h) * a.nblk + blk];
+#pragma unroll 4
+  for (int r = 0; r < RPW; ++r) {
+    const int n = blk * 128 + warp * RPW + r;  // uniform over the warp
+    if (n >= a.N) break;
+    const size_t off = ((static_cast<size_t>(b) * a.N + n) * a.H + h) * D + lane * E;
+    float v[E];
+    if constexpr (E == 4) {
+      const uint32_t c = __ldg(reinterpret_cast<const uint32_t*>(a.codes + off));
+      const uint32_t lo = e4m3x2_to_f16x2(static_cast<uint16_t>(c & 0xffffu));
+      const uint32_t hi = e4m3x2_to_f16x2(static_cast<uint16_t>(c >> 16));
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+      v[0] = f0.x * s;
+      v[1] = f0.y * s;
+      v[2] = f1.x * s;
+      v[3] = f1.y * s;
+    } else {
+      const uint16_t c = __ldg(reinterpret_cast<const uint16_t*>(a.codes + off));
+      const uint32_t w = e4m3x2_to_f16x2(c);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w));
+      v[0] = f0.x * s;
+      v[1] = f0.y * s;
+    }
+    if (a.unrotate) {  // uniform over the grid
+#pragma unroll
+      for (int w = 1; w < E; w *= 2) {
+        float t[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) t[e] = (e & w) ? v[e - w] - v[e] : v[e] + v[e + w];
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = t[e];
+      }
+#pragma unroll
+      for (int lw = 1; lw < 32; lw *= 2) {
+        const bool upper = lane & lw;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float p = __shfl_xor_sync(0xffffffffu, v[e], lw);
+          v[e] = upper ? p - v[e] : v[e] + p;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) v[e] = v[e] * a.rscale;
+    }
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.x) + off;
+    if constexpr (E == 4)
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    else
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(v[0], v[1]);
+  }
+}
+
 }  // namespace fa

@@ -1,0 +1,69 @@
+"""GPU parity of the fp8 backward pieces (through the C-ABI).
+
+* fa_fp8_dequantize: bit-identical to the oracle's float32 steps
+  (code * scale, with the inverse rotation the butterflies and the
+  1/sqrt(d) multiply) rounded to nearest-even bf16, d = 64 and 128, ragged N,
+  with and without the rotation.
+* attention_bwd_fp8 (dequantise, then the bf16 backward with the fp8
+  forward's O and LSE): dQ, dK, dV against the oracle's gradient of exact
+  attention on the dequantised fp32 values, with the bf16 backward bound
+  (relative RMS <= 1e-2), causal or not, rotated Q/K or not.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+G_REL_RMS = 1e-2
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import io_aware_exact_27_b200 as m
+    return m
+
+
+@pytest.mark.parametrize("unrotate", [False, True])
+@pytest.mark.parametrize("B,N,H,d", [(1, 300, 3, 128), (2, 129, 2, 64), (1, 1, 1, 128)])
+def test_dequantize_bit_exact(fa, B, N, H, d, unrotate):
+    x = synth.qkv_bf16(7 + N, B, N, H, H, d)[0].cuda()
+    codes, scales = fa.quantize_fp8(x, rotate=unrotate)
+    y = fa.dequantize_fp8(codes, scales, unrotate=unrotate)
+    torch.cuda.synchronize()
+    want = oracle.dequantize_f32(codes.cpu().float().numpy(), scales.cpu().numpy(), unrotate=unrotate)
+    want_bf16 = torch.from_numpy(want).to(torch.bfloat16)
+    assert torch.equal(y.cpu(), want_bf16)
+
+
+@pytest.mark.parametrize("rotated", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_backward_matches_oracle(fa, causal, rotated):
+    B, N, H, d = 1, 1000, 4, 128
+    q, k, v, do = synth.qkv_bf16(40 + int(causal) + 2 * int(rotated), B, N, H, H, d, with_dout=True)
+    dev = torch.device("cuda")
+    q8, qs = fa.quantize_fp8(q.to(dev), rotate=rotated)
+    k8, ks = fa.quantize_fp8(k.to(dev), rotate=rotated)
+    v8, vs = fa.quantize_fp8(v.to(dev), rotate=False)
+    scale = 1 / math.sqrt(d)
+    o, lse = fa.attention_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, scale=scale)
+    dq, dk, dv = fa.attention_bwd_fp8(q8, k8, v8, qs, ks, vs, o, lse, do.to(dev), causal=causal, scale=scale,
+                                      rotated=rotated)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    deq = [oracle.dequantize_f32(c.cpu().float().numpy(), s.cpu().numpy(), unrotate=u)
+           for c, s, u in ((q8, qs, rotated), (k8, ks, rotated), (v8, vs, False))]
+    want = oracle.attn_bwd(*deq, do, causal, scale)
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        gn = g.double().cpu().numpy()
+        assert np.all(np.isfinite(gn)), name
+        rr = oracle.rel_rms(gn, w)
+        assert rr <= G_REL_RMS, f"{name} rel-RMS {rr}"
