@@ -897,6 +897,21 @@ def run_fp8(args):
     def forward():
         fa.fa_fwd_fp8(codes[0], codes[1], codes[2], scl[0], scl[1], scl[2], o, lse, B, H, H, N, d, 1, scale, sptr)
 
+    # the training step's backward, timed apart: dequantise Q, K (rotation
+    # undone) and V, then the bf16 backward with the fp8 forward's O and LSE
+    import synth
+    do = synth.qkv_bf16(rank + 200, B, N, H, H, d, with_dout=True)[3].to(dev)
+    deq = [torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    grads = [torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    ws_bytes = fa.fa_bwd_workspace_size(B * N, B, H, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def backward():
+        for i, rot in enumerate((True, True, False)):
+            fa.fa_fp8_dequantize(codes[i], scl[i], deq[i], B, N, H, d, int(rot), sptr)
+        fa.fa_bwd(deq[0], deq[1], deq[2], o, lse, do, grads[0], grads[1], grads[2], ws, ws_bytes, B, H, H, N, d, 1,
+                  scale, sptr)
+
     # error against fp64 attention on the unquantised fp32 values (sampled rows)
     rows = fp8_sample_rows(N)
     rows_h = np.tile(rows[None, :], (H, 1))
@@ -912,6 +927,7 @@ def run_fp8(args):
     for _ in range(args.warmup):
         quantize()
         forward()
+        backward()
     torch.cuda.synchronize(dev)
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error during warm-up")
@@ -934,6 +950,16 @@ def run_fp8(args):
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     f_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     tot_ms = (q_ms + f_ms) * args.steps
+    bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for b0, b1 in bev:
+        flush.zero_()
+        b0.record(stream)
+        backward()
+        b1.record(stream)
+    torch.cuda.synchronize(dev)
+    b_ms = sum(b0.elapsed_time(b1) for b0, b1 in bev) / args.steps
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error in the backward")
     if pg:
         t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -998,7 +1024,10 @@ def run_fp8(args):
             "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic", "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
-            "gpu_launches": 4 * args.steps}
+            "gpu_launches": 4 * args.steps,
+            "backward": {"ms": b_ms, "tflops": 2.5 * flops / (b_ms * 1e-3) / 1e12,
+                         "note": "fa_fp8_dequantize x3 (Q, K unrotated) + fa_bwd with the fp8 forward's O and LSE, "
+                                 "timed apart, per GPU; flops 2.5x the forward's"}}
     print(json.dumps(line), flush=True)
     return 0
 
