@@ -79,24 +79,40 @@ def peaks():
     return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+# the device source file that defines each profiled kernel
+KERNEL_HEADER = {"fa_fwd_sm100_kernel": "fa_fwd_kernel.cuh", "fa_bwd_dkdv_kernel": "fa_bwd_kernel.cuh",
+                 "fa_bwd_dq_kernel": "fa_bwd_kernel.cuh", "fa_decode_kernel": "fa_decode_kernel.cuh"}
+
+
+def kernel_source_hash(kernel):
+    """Hash of a kernel's device code: its header and every header it includes
+    (followed transitively). The host launcher is not part of it: a change of
+    a kernel's launch configuration there must be re-captured by hand."""
+    import re
     csrc = os.path.join(ROOT, "io_aware_exact_27_b200", "csrc")
+    todo, seen = [KERNEL_HEADER[kernel]], []
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.append(f)
+        todo += re.findall(r'^#include "([^"]+)"', open(os.path.join(csrc, f)).read(), flags=re.M)
     h = hashlib.sha256()
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in sorted(seen):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
-    when the kernel sources changed since those counters were taken."""
+    when the kernel's device sources changed since those counters were taken."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kernel not in KERNEL_HEADER:
         return None
     j = json.load(open(p))
     e = j.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
