@@ -623,16 +623,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             break;
           }
           if (lane == 0) {
-            const uint32_t bar = smem_u32(&sm.qo_full[slot]);
+            // a step's Q and dO tiles and the query tile's LSE2 and D all
+            // complete on the Q slot's barrier (Q sits in the even ring
+            // slots): one wait covers the step for the MMA issuer, where
+            // every mbarrier wait costs tensor-pipe time
+            const uint32_t bar = smem_u32(&sm.qo_full[w == 0 ? slot : (slot + STAGES - 1) % STAGES]);
             if (w == 0) {
-              // the query tile's LSE2 and D ride on the Q tile's barrier
               float* vec = sm.vec[(qo_prod / 2) % (STAGES / 2)][0];
               const size_t wbase = static_cast<size_t>(hq) * args.ws_stride + ws_offset(un.tok0, un.seq) + qi * kBM;
-              mbar_expect_tx(bar, Smem::kTileBytes + 1024);
+              mbar_expect_tx(bar, 2 * Smem::kTileBytes + 1024);
               bulk_load(smem_u32(vec), args.lse2 + wbase, 512, bar);
               bulk_load(smem_u32(vec + 128), args.dvec + wbase, 512, bar);
-            } else {
-              mbar_expect_tx(bar, Smem::kTileBytes);
             }
             load_tile<D>(smem_u32(sm.qo[slot]), w == 0 ? &tm_q : &tm_do, bar, hq, un.tok0 + qi * kBM);
           }
@@ -669,7 +670,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         uint32_t slotO = (qo_cons + 1) % STAGES;
         issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[slotQ]));
         tc_commit(smem_u32(&sm.s_full));
-        if (!(ok = wait(&sm.qo_full[slotO], ((qo_cons + 1) / STAGES) & 1, 72))) break;
         issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[slotO]));
         tc_commit(smem_u32(&sm.dp_full));
         if (nsteps == 1) tc_commit(smem_u32(&sm.kv_empty));  // last reads of K and V issued
@@ -696,7 +696,6 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           issue_ts_split<D>(tDK, tDP, smem_u32(sm.qo[slotQ]), st > 0);
           tc_commit(smem_u32(&sm.qo_empty[slotQ]));  // Q_st: last use
           if (has_next) {
-            if (!(ok = wait(&sm.qo_full[nO], ((qo_cons + 1) / STAGES) & 1, 77))) break;
             issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[nO]));
             tc_commit(smem_u32(&sm.dp_full));
             // K and V are last read by this unit's final S^T and dP^T: release
@@ -839,8 +838,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   tc_fence_before();
   __syncthreads();
   if (sm.abort && warp == 8 && lane == 0) {
+    // (only the Q slots' barriers complete: a step's dO load counts on its Q slot)
     for (uint32_t i = (prod_issued > STAGES ? prod_issued - STAGES : 0); i < prod_issued; ++i)
-      mbar_wait(smem_u32(&sm.qo_full[i % STAGES]), (i / STAGES) & 1, nullptr, args.timeout_ns);
+      if ((i & 1) == 0) mbar_wait(smem_u32(&sm.qo_full[i % STAGES]), (i / STAGES) & 1, nullptr, args.timeout_ns);
     if (kv_issued > 0) mbar_wait(smem_u32(&sm.kv_full), (kv_issued - 1) & 1, nullptr, args.timeout_ns);
   }
   __syncthreads();
