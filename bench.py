@@ -1168,7 +1168,7 @@ def run_blocksparse(args):
     # dense causal backward beside it); flops 2.5x the forward's (five GEMMs)
     do = synth.qkv_bf16(rank + 100, B, N, Hq, Hkv, d, with_dout=True)[3].to(dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_bytes = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+    ws_bytes = fa.fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d)  # >= the dense backward's
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     o_bs = torch.empty_like(q)
     lse_bs = torch.empty_like(lse)

@@ -226,13 +226,24 @@ fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, cons
  * exactly as given to fa_fwd_blocksparse (DEVICE uint8 [Hq][nb][nb]); o and
  * lse are that call's outputs (a row with lse = -inf gets dQ = 0). dQ units
  * visit only the key blocks their query tile sees; dK/dV units only the
- * (query head, query tile) steps that see their key tile; a tile that sees
- * nothing writes zeros. Deterministic. NULL mask: FA_ERR_INVALID_ARG.
+ * (query head, query tile) steps that see their key tile, following a work
+ * plan made on the device: a unit more than twice the average unit long (a
+ * key block every query block sees) is split into chunks of about the
+ * average, whose fp32 partial sums are added in chunk order afterwards. A
+ * tile that sees nothing writes zeros. Deterministic.
+ *   workspace: ws_bytes >= fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d)
+ *   (the two vectors of fa_bwd plus the plan and four partial [128][d] fp32
+ *   pairs per SM of the current device), 256-byte aligned; FA_ERR_WORKSPACE
+ *   otherwise. NULL mask: FA_ERR_INVALID_ARG.
  */
 fa_status_t fa_bwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask,
                                const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
                                void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
                                float scale, void* stream);
+
+/* Workspace bytes fa_bwd_blocksparse needs on the current device; 0 for
+ * invalid sizes or when no device is available. */
+size_t fa_bwd_blocksparse_workspace_size(int B, int Hq, int Hkv, int N, int d);
 
 /*
  * Block-scaled e4m3 inputs for fa_fwd_fp8, with optional incoherent

@@ -58,6 +58,8 @@ for _name, _args in _SIGS.items():
     getattr(_lib, _name).restype = _I
 _lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_size.restype = _Z
+_lib.fa_bwd_blocksparse_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+_lib.fa_bwd_blocksparse_workspace_size.restype = _Z
 _lib.fa_fwd_kvcache_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.fa_fwd_kvcache_workspace_size.restype = _Z
 _lib.fa_fwd_kvcache_num_splits.argtypes = [_I, _I, _I, _I]
@@ -128,6 +130,10 @@ def fa_bwd_workspace_size(tokens, nseq, Hq, d) -> int:
     return int(_lib.fa_bwd_workspace_size(tokens, nseq, Hq, d))
 
 
+def fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d) -> int:
+    return int(_lib.fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d))
+
+
 def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N, d, causal, scale, stream=None):
     _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                        _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)),
@@ -175,7 +181,7 @@ def attention_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, causal=False, s
     import torch
     B, N, Hq, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_bytes = fa_bwd_workspace_size(B * N, B, Hq, d)
+    ws_bytes = fa_bwd_blocksparse_workspace_size(B, Hq, k.shape[2], N, d)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     fa_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), B, Hq,

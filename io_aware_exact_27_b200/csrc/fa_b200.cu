@@ -204,6 +204,30 @@ size_t vec_bytes(int tokens, int nseq, int Hq) {
   return (b + 255) & ~size_t(255);
 }
 
+// Block-sparse backward: the dK/dV work plan and the split units' partial
+// sums follow the two workspace vectors. units = B * Hkv * ceil(N/128);
+// partial slots: 4 per SM (the plan leaves units unsplit beyond that).
+struct SparsePlanLayout {
+  long long units, max_slots, max_items, max_steps;
+  size_t plan_off, nbuf_off, sbase_off, steps_off, part_off, total;
+};
+SparsePlanLayout sparse_plan_layout(size_t base, int B, int Hq, int Hkv, int N, int d, int sms) {
+  SparsePlanLayout L{};
+  const long long nqb = (N + 127) / 128;
+  L.units = static_cast<long long>(B) * Hkv * nqb;
+  L.max_steps = L.units * (Hq / Hkv) * nqb;  // every (query head, query tile) of every unit
+  L.max_slots = 4LL * sms;
+  L.max_items = L.units + L.max_slots;
+  const size_t plan_ints = 4 + 4 * static_cast<size_t>(L.max_items) + 4 * static_cast<size_t>(L.max_slots);
+  L.plan_off = (base + 255) & ~size_t(255);
+  L.nbuf_off = (L.plan_off + plan_ints * sizeof(int) + 255) & ~size_t(255);
+  L.sbase_off = (L.nbuf_off + static_cast<size_t>(L.units) * sizeof(int) + 255) & ~size_t(255);
+  L.steps_off = (L.sbase_off + static_cast<size_t>(L.units) * sizeof(int) + 255) & ~size_t(255);
+  L.part_off = (L.steps_off + static_cast<size_t>(L.max_steps) * sizeof(int) + 255) & ~size_t(255);
+  L.total = L.part_off + static_cast<size_t>(L.max_slots) * 2 * 128 * d * sizeof(float);
+  return L;
+}
+
 template <int D, bool SPARSE = false>
 fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* dout,
                        fa::BwdArgs a, long long units_dq, long long units_dkdv, int parts, cudaStream_t stream) {
@@ -243,7 +267,34 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   }
   fa::BwdArgs akv = a;
   akv.num_units = static_cast<int>(units_dkdv);
-  const int g1 = static_cast<int>(units_dkdv < ds->sms ? units_dkdv : ds->sms);
+  long long work_dkdv = units_dkdv;  // dense: units; block-sparse: an upper bound of the planned items
+  if (SPARSE) work_dkdv = a.plan_max_items;
+  const int g1 = static_cast<int>(work_dkdv < ds->sms ? work_dkdv : ds->sms);
+  // dK/dV on `stream`; block-sparse: the work plan (one CTA) before it and
+  // the sums of the split units' partials after it
+  auto run_dkdv = [&]() -> bool {
+    if (SPARSE) {
+      // the per-CTA share counts one CTA per unit at most: units are only
+      // split when far longer than the others, never to widen the grid
+      const int share_grid = static_cast<int>(units_dkdv < g1 ? units_dkdv : g1);
+      fa::fa_bwd_plan_count_kernel<<<static_cast<int>((units_dkdv + 7) / 8), 256, 0, stream>>>(
+          a, static_cast<int>(units_dkdv), a.plan_nbuf);
+      if (cudaGetLastError() != cudaSuccess) return false;
+      fa::fa_bwd_plan_kernel<<<1, fa::kPlanThreads, 0, stream>>>(a, static_cast<int>(units_dkdv), share_grid,
+                                                                 a.plan_max_slots, a.plan_nbuf);
+      if (cudaGetLastError() != cudaSuccess) return false;
+      fa::fa_bwd_plan_steps_kernel<<<static_cast<int>((units_dkdv + 7) / 8), 256, 0, stream>>>(
+          a, static_cast<int>(units_dkdv));
+      if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
+    if (cudaGetLastError() != cudaSuccess) return false;
+    if (SPARSE) {
+      fa::fa_bwd_reduce_kernel<D><<<ds->sms, 256, 0, stream>>>(a);
+      if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    return true;
+  };
   fa::BwdArgs aq = a;
   aq.num_units = static_cast<int>(units_dq);
   const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
@@ -261,8 +312,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
     }
     if (cudaEventRecord(ds->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ds->side, ds->fork, 0) != cudaSuccess)
       return FA_ERR_CUDA;
-    kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (!run_dkdv()) return FA_ERR_CUDA;
     kdq<<<g2, fa::kThreadsBwd, smem_dq, ds->side>>>(tq, tk, tv, tdo, aq);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (cudaEventRecord(ds->join, ds->side) != cudaSuccess || cudaStreamWaitEvent(stream, ds->join, 0) != cudaSuccess)
@@ -270,8 +320,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
     return FA_OK;
   }
   if (parts & FA_BWD_DKDV) {
-    if (g1 > 0) kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (g1 > 0 && !run_dkdv()) return FA_ERR_CUDA;
   }
   if (parts & FA_BWD_DQ) {
     if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
@@ -294,6 +343,12 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < 2 * vb) return FA_ERR_WORKSPACE;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
+  SparsePlanLayout L{};
+  if (block_mask != nullptr) {
+    L = sparse_plan_layout(2 * vb, nseq, Hq, Hkv, N, d, ds->sms);
+    if (ws_bytes < L.total) return FA_ERR_WORKSPACE;
+    if (L.max_items > INT32_MAX / 4 || L.max_steps > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  }
   fa::BwdArgs a{};
   a.o = o;
   a.dout = dout;
@@ -332,6 +387,16 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   if (parts <= 0 || parts > FA_BWD_ALL) return FA_ERR_INVALID_ARG;
   a.block_mask = block_mask;
   a.nqb = static_cast<int>(nt);
+  if (block_mask != nullptr) {
+    char* w = static_cast<char*>(workspace);
+    a.plan = reinterpret_cast<int*>(w + L.plan_off);
+    a.plan_nbuf = reinterpret_cast<int*>(w + L.nbuf_off);
+    a.plan_sbase = reinterpret_cast<int*>(w + L.sbase_off);
+    a.plan_steps = reinterpret_cast<int*>(w + L.steps_off);
+    a.partials = reinterpret_cast<float*>(w + L.part_off);
+    a.plan_max_items = static_cast<int>(L.max_items);
+    a.plan_max_slots = static_cast<int>(L.max_slots);
+  }
   if (block_mask != nullptr)
     return d == 128 ? launch_bwd<128, true>(ds, q, k, v, dout, a, udq, ukv, parts, s)
                     : launch_bwd<64, true>(ds, q, k, v, dout, a, udq, ukv, parts, s);
@@ -500,6 +565,14 @@ size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
   (void)d;
   if (tokens <= 0 || Hq <= 0 || nseq < 0) return 0;
   return 2 * vec_bytes(tokens, nseq, Hq);
+}
+
+size_t fa_bwd_blocksparse_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (B <= 0 || N <= 0 || Hq <= 0 || Hkv <= 0 || (d != 64 && d != 128)) return 0;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return 0;
+  DeviceState* ds = nullptr;
+  if (device_state(&ds) != FA_OK) return 0;
+  return sparse_plan_layout(2 * vec_bytes(B * N, B, Hq), B, Hq, Hkv, N, d, ds->sms).total;
 }
 
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,

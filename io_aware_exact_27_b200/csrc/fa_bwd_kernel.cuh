@@ -55,6 +55,18 @@ struct BwdArgs {
   // block-sparse: [Hq][nqb][nqb] uint8 as for the forward; null = dense
   const uint8_t* block_mask;
   int nqb;
+  // block-sparse dK/dV work plan (written by fa_bwd_plan_kernel): plan[0] =
+  // items, plan[1] = split units; from int 4 on, plan_max_items items of 4
+  // ints (unit, first visible step, steps, partial slot or -1), then the
+  // split units (unit, first slot, chunks, 0). partials: [slot][dV, dK]
+  // [128 rows][D] fp32 sums of a split unit's chunks.
+  int* plan;
+  float* partials;
+  int plan_max_items;
+  int plan_max_slots;
+  int* plan_nbuf;   // visible steps per unit
+  int* plan_sbase;  // first entry of each unit's steps in plan_steps
+  int* plan_steps;  // every unit's visible steps, in order (unit after unit)
 };
 
 // ------------------------------------------------------------------ pre
@@ -69,15 +81,27 @@ __device__ __forceinline__ int ws_offset(int tok0, int seq) { return ((tok0 + 3)
 // Block-sparse backward (the forward's mask): key block kb visible to query
 // block qb of query head hq. A dQ unit (query tile qt of head h) walks the key
 // blocks it sees; a dK/dV unit (key tile kb of kv head hk) walks the (query
-// head of the group, query tile) steps that see it. A unit that sees none
-// still runs one block / step, every score masked (zero gradient), so that
-// every role runs the same pipeline.
+// head of the group, query tile) steps that see it, read from the step lists
+// of the work plan (see fa_bwd_plan_kernel). A unit that sees none still runs
+// one block / step, every score masked (zero gradient), so that every role
+// runs the same pipeline.
 __device__ __forceinline__ bool bwd_block_on(const BwdArgs& a, int hq, int qb, int kb) {
   return __ldg(a.block_mask + (static_cast<size_t>(hq) * a.nqb + qb) * a.nqb + kb) != 0;
 }
+// Bit e set when key block base + e (< jend) is seen by query tile qt of
+// head h: eight independent loads per round (one round trip for eight).
+__device__ __forceinline__ uint32_t dq_blocks_on8(const BwdArgs& a, int h, int qt, int base, int jend) {
+  const uint8_t* r = a.block_mask + (static_cast<size_t>(h) * a.nqb + qt) * a.nqb;
+  uint32_t on = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) on |= (base + e < jend && __ldg(r + base + e) != 0) ? (1u << e) : 0u;
+  return on;
+}
 __device__ __forceinline__ int dq_next_block(const BwdArgs& a, int h, int qt, int j, int jend) {
-  for (int jj = j + 1; jj < jend; ++jj)
-    if (bwd_block_on(a, h, qt, jj)) return jj;
+  for (int base = j + 1; base < jend; base += 8) {
+    const uint32_t on = dq_blocks_on8(a, h, qt, base, jend);
+    if (on) return base + __ffs(on) - 1;
+  }
   return jend;
 }
 __device__ __forceinline__ int dq_first_block(const BwdArgs& a, int h, int qt, int jend) {
@@ -86,30 +110,9 @@ __device__ __forceinline__ int dq_first_block(const BwdArgs& a, int h, int qt, i
 }
 __device__ __forceinline__ int dq_count_blocks(const BwdArgs& a, int h, int qt, int jend) {
   int n = 0;
-  for (int j = dq_next_block(a, h, qt, -1, jend); j < jend; j = dq_next_block(a, h, qt, j, jend)) ++n;
+  for (int base = 0; base < jend; base += 8) n += __popc(dq_blocks_on8(a, h, qt, base, jend));
   return n > 0 ? n : 1;
 }
-// dK/dV step st of a unit: query head hk*group + st / nqt, query tile i0 + st % nqt
-__device__ __forceinline__ int kv_next_step(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb, int st,
-                                            int nsteps) {
-  for (int s2 = st + 1; s2 < nsteps; ++s2)
-    if (bwd_block_on(a, hk * group + s2 / nqt, i0 + s2 % nqt, kb)) return s2;
-  return nsteps;
-}
-__device__ __forceinline__ int kv_first_step(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb,
-                                             int nsteps) {
-  const int s2 = kv_next_step(a, hk, group, nqt, i0, kb, -1, nsteps);
-  return s2 < nsteps ? s2 : 0;
-}
-__device__ __forceinline__ int kv_count_steps(const BwdArgs& a, int hk, int group, int nqt, int i0, int kb,
-                                              int nsteps) {
-  int n = 0;
-  for (int s2 = kv_next_step(a, hk, group, nqt, i0, kb, -1, nsteps); s2 < nsteps;
-       s2 = kv_next_step(a, hk, group, nqt, i0, kb, s2, nsteps))
-    ++n;
-  return n > 0 ? n : 1;
-}
-
 // Workspace entry r = (head h, index i) -> the token it holds, or -1 for a
 // gap / trailing filler entry: the last sequence whose block starts at or
 // before i (binary search over the sequence starts).
@@ -581,23 +584,35 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     nqt = nq - i0;
     return group * nqt;
   };
-  auto first_step = [&](const Unit& un, int i0, int nqt, int nsteps) {
-    return SPARSE ? kv_first_step(args, un.h, group, nqt, i0, un.qb2, nsteps) : 0;
+  // work item w: block-sparse, the planned (unit, position of its first step
+  // in the planned step list or -1 for a key tile nothing sees, steps,
+  // partial slot or -1); dense, unit w whole
+  const int nwork = SPARSE ? __ldg(args.plan) : num_units;
+  auto work_of = [&](int w) -> int4 {
+    if constexpr (SPARSE)
+      return __ldg(reinterpret_cast<const int4*>(args.plan) + 1 + w);
+    else
+      return make_int4(w, 0, 0, -1);
   };
-  auto next_step = [&](const Unit& un, int i0, int nqt, int st, int nsteps) {
-    return SPARSE ? kv_next_step(args, un.h, group, nqt, i0, un.qb2, st, nsteps) : st + 1;
+  // step v of an item
+  auto step_of = [&](const int4& wk, int v) -> int {
+    if constexpr (SPARSE)
+      return wk.y < 0 ? 0 : __ldg(args.plan_steps + wk.y + v);
+    else
+      return v;
   };
 
   if (warp == 8) {
     uint32_t qo_prod = 0, it = 0;
     bool ok = true;
     for (int rnd = 0; ok; ++rnd, ++it) {
-      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
-      if (u >= num_units) break;
-      const Unit un = decode_unit(sched, u);
+      const int w = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (w >= nwork) break;
+      const int4 wk = work_of(w);
+      const Unit un = decode_unit(sched, wk.x);
       int i0, nqt;
       const int nsteps = unit_steps(un, i0, nqt);
-      const int nvis = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nsteps) : nsteps;
+      const int nvis = SPARSE ? wk.z : nsteps;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.kv_empty), (it & 1) ^ 1, abort, args.timeout_ns));
       if (!ok) {
         if (lane == 0) report_error(args.status, kStatusTimeout, 60);
@@ -610,8 +625,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         load_tile<D>(smem_u32(sm.v), &tm_v, bar, un.h, un.tok0 + un.qb2 * kBN);
       }
       kv_issued = it + 1;
-      int st = first_step(un, i0, nqt, nsteps);
-      for (int v = 0; v < nvis && ok; ++v, st = next_step(un, i0, nqt, st, nsteps)) {
+      for (int v = 0; v < nvis && ok; ++v) {
+        const int st = step_of(wk, v);
         const int hq = un.h * group + st / nqt;
         const int qi = i0 + st % nqt;
         for (int w = 0; w < 2; ++w) {
@@ -656,12 +671,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         return true;
       };
       for (int rnd = 0; ok; ++rnd, ++it) {
-        const int u = unit_of(rnd, blockIdx.x, gridDim.x);
-        if (u >= num_units) break;
-        const Unit un = decode_unit(sched, u);
+        const int w = unit_of(rnd, blockIdx.x, gridDim.x);
+        if (w >= nwork) break;
+        const int4 wk = work_of(w);
+        const Unit un = decode_unit(sched, wk.x);
         int i0, nqt;
         const int nall = unit_steps(un, i0, nqt);
-        const int nsteps = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nall) : nall;  // visited
+        const int nsteps = SPARSE ? wk.z : nall;  // visited
         if (!(ok = wait(&sm.kv_full, it & 1, 70))) break;
         const uint32_t ka = smem_u32(sm.k), va = smem_u32(sm.v);
         // prologue: S^T(0), dP^T(0)
@@ -723,19 +739,20 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     uint32_t sc = 0, dpc = 0, it = 0, vstep = 0;
     bool ok = true;
     for (int rnd = 0; ok; ++rnd, ++it) {
-      const int u = unit_of(rnd, blockIdx.x, gridDim.x);
-      if (u >= num_units) break;
-      const Unit un = decode_unit(sched, u);
+      const int w = unit_of(rnd, blockIdx.x, gridDim.x);
+      if (w >= nwork) break;
+      const int4 wk = work_of(w);
+      const Unit un = decode_unit(sched, wk.x);
       int i0, nqt;
       const int nsteps = unit_steps(un, i0, nqt);
-      const int nvis = SPARSE ? kv_count_steps(args, un.h, group, nqt, i0, un.qb2, nsteps) : nsteps;
+      const int nvis = SPARSE ? wk.z : nsteps;
       const int key = un.qb2 * kBN + r_in_tile;  // key row within the sequence
       const bool valid = key < un.n;
-      int st = first_step(un, i0, nqt, nsteps);
-      for (int v = 0; v < nvis; ++v, ++vstep, st = next_step(un, i0, nqt, st, nsteps)) {
+      for (int v = 0; v < nvis; ++v, ++vstep) {
+        const int st = step_of(wk, v);
         const int qi = i0 + st % nqt;
-        // block-sparse: the forced visit of a unit that no query tile sees
-        const bool off = SPARSE && !bwd_block_on(args, un.h * group + st / nqt, qi, un.qb2);
+        // block-sparse: the forced visit of a key tile that no query tile sees
+        const bool off = SPARSE && wk.y < 0;
         const float* vec = sm.vec[vstep % (STAGES / 2)][0];
         const int q0 = qi * kBM + half * 64;  // first query column of this half
         // the producer stored this step's LSE2/D before arriving on the Q
@@ -817,6 +834,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         for (int c = 0; c < HC; c += 32) {
           uint32_t orr[32];
           tmem_ld32(src + c, orr);
+          if (SPARSE && wk.w >= 0) {
+            // a chunk of a split unit: its fp32 sums to its partial slot
+            float4* prow = reinterpret_cast<float4*>(args.partials +
+                                                     ((static_cast<size_t>(wk.w) * 2 + which) * kBN + r_in_tile) * D +
+                                                     half * HC + c);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              prow[t] = make_float4(__uint_as_float(orr[4 * t]), __uint_as_float(orr[4 * t + 1]),
+                                    __uint_as_float(orr[4 * t + 2]), __uint_as_float(orr[4 * t + 3]));
+            continue;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t)
@@ -848,6 +876,182 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ block-sparse dK/dV plan
+// With a block mask the dK/dV units can be very uneven (a key block every
+// query block sees, e.g. a global first block, makes a unit group x nqb steps
+// long against a handful for the others), and the CTA that holds such a unit
+// bounds the kernel. fa_bwd_plan_count_kernel counts every unit's visible
+// steps n_u; one CTA then takes
+// a chunk length L = max(16, min(ceil(sum n / grid), ceil(sum n / units)))
+// (the average unit, or the per-CTA share when there are fewer units than
+// CTAs); a unit with n_u > 2L becomes ceil(n_u / L) chunks of (nearly) equal
+// step counts, so that the items dealt round-robin to the CTAs are of about
+// equal size. A split unit's chunks write fp32 partial dK/dV into their own
+// slots, which fa_bwd_reduce_kernel sums in chunk order (deterministic). The
+// slots are bounded (max_slots): a run of units whose chunks would not fit
+// stays unsplit. A dense or causal mask never splits (no unit is twice the
+// average).
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMinChunk = 16;
+// Visible steps of every dK/dV unit (at least 1, the forced visit of a unit
+// nothing sees), one warp per unit: the lanes test 32 steps at a time.
+__global__ void __launch_bounds__(256) fa_bwd_plan_count_kernel(const BwdArgs a, int units, int* nbuf) {
+  const int u = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (u >= units) return;  // uniform over the warp
+  const int group = a.Hq / a.Hkv;
+  const int nlevels = (a.N + 127) / 128;
+  const SeqSched sched{nullptr, a.nseq, a.N, a.Hkv, a.causal, nlevels, nullptr, 7};
+  const Unit un = decode_unit(sched, u);
+  const int i0 = a.causal ? un.qb2 : 0;
+  const int nqt = (un.n + 127) / 128 - i0;
+  int n = 0;
+  for (int base = 0; base < group * nqt; base += 32) {
+    const int st = base + lane;
+    const bool on = st < group * nqt && bwd_block_on(a, un.h * group + st / nqt, i0 + st % nqt, un.qb2);
+    n += __popc(__ballot_sync(0xffffffffu, on));
+  }
+  if (lane == 0) nbuf[u] = n;
+}
+
+// Writes the visible steps of unit u at plan_steps[plan_sbase[u] ...], in
+// step order (one warp per unit: ballot, then each set lane's rank).
+__global__ void __launch_bounds__(256) fa_bwd_plan_steps_kernel(const BwdArgs a, int units) {
+  const int u = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (u >= units) return;  // uniform over the warp
+  const int group = a.Hq / a.Hkv;
+  const int nlevels = (a.N + 127) / 128;
+  const SeqSched sched{nullptr, a.nseq, a.N, a.Hkv, a.causal, nlevels, nullptr, 7};
+  const Unit un = decode_unit(sched, u);
+  const int i0 = a.causal ? un.qb2 : 0;
+  const int nqt = (un.n + 127) / 128 - i0;
+  int pos = a.plan_sbase[u];
+  for (int base = 0; base < group * nqt; base += 32) {
+    const int st = base + lane;
+    const bool on = st < group * nqt && bwd_block_on(a, un.h * group + st / nqt, i0 + st % nqt, un.qb2);
+    const uint32_t bal = __ballot_sync(0xffffffffu, on);
+    if (on) a.plan_steps[pos + __popc(bal & ((1u << lane) - 1u))] = st;
+    pos += __popc(bal);
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) fa_bwd_plan_kernel(const BwdArgs a, int units, int grid, int max_slots,
+                                                                   const int* nbuf) {
+  __shared__ long long red[kPlanThreads];
+  __shared__ int scan_items[kPlanThreads], scan_slots[kPlanThreads], scan_splits[kPlanThreads];
+  __shared__ int scan_steps[kPlanThreads];
+  __shared__ unsigned char nosplit[kPlanThreads];
+  const int tid = threadIdx.x;
+  long long local = 0;
+  for (int u = tid; u < units; u += kPlanThreads) local += nbuf[u];
+  red[tid] = local;
+  __syncthreads();
+  for (int off = kPlanThreads / 2; off > 0; off >>= 1) {
+    if (tid < off) red[tid] += red[tid + off];
+    __syncthreads();
+  }
+  const long long total = red[0];
+  const long long share = (total + grid - 1) / grid, avg = (total + units - 1) / units;
+  const long long L = max(static_cast<long long>(kPlanMinChunk), min(share, avg));
+  auto chunks_of = [&](int n) -> int { return n > 2 * L ? static_cast<int>((n + L - 1) / L) : 1; };  // n >= 0
+  // each thread takes a contiguous segment of units, in unit order
+  const int seg = (units + kPlanThreads - 1) / kPlanThreads;
+  const int u0 = min(units, tid * seg), u1 = min(units, u0 + seg);
+  int items = 0, slots = 0, splits = 0, steps = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int c = chunks_of(nbuf[u]);
+    items += c;
+    steps += nbuf[u];
+    if (c > 1) {
+      slots += c;
+      ++splits;
+    }
+  }
+  scan_items[tid] = items;
+  scan_slots[tid] = slots;
+  scan_splits[tid] = splits;
+  scan_steps[tid] = steps;
+  __syncthreads();
+  if (tid == 0) {  // exclusive scans in segment (= unit) order; segments over the slot budget stay unsplit
+    int ai = 0, as = 0, ap = 0, at = 0;
+    for (int i = 0; i < kPlanThreads; ++i) {
+      const int xt = scan_steps[i];
+      scan_steps[i] = at;
+      at += xt;
+      int xi = scan_items[i], xs = scan_slots[i], xp = scan_splits[i];
+      nosplit[i] = as + xs > max_slots;
+      if (nosplit[i]) {
+        xi = max(0, min(units, (i + 1) * seg) - min(units, i * seg));
+        xs = 0;
+        xp = 0;
+      }
+      scan_items[i] = ai;
+      scan_slots[i] = as;
+      scan_splits[i] = ap;
+      ai += xi;
+      as += xs;
+      ap += xp;
+    }
+    a.plan[0] = ai;
+    a.plan[1] = ap;
+  }
+  __syncthreads();
+  int4* item = reinterpret_cast<int4*>(a.plan) + 1;
+  int4* split = item + a.plan_max_items;
+  int wi = scan_items[tid], ws = scan_slots[tid], wp = scan_splits[tid], wt = scan_steps[tid];
+  for (int u = u0; u < u1; ++u) {
+    const int n = nbuf[u];
+    a.plan_sbase[u] = wt;
+    if (n == 0) {  // nothing sees this key tile: one forced step, every score masked
+      item[wi++] = make_int4(u, -1, 1, -1);
+      continue;
+    }
+    const int c = nosplit[tid] ? 1 : chunks_of(n);
+    const int per = (n + c - 1) / c;
+    for (int k = 0; k < c; ++k)
+      item[wi++] = make_int4(u, wt + k * per, min(per, n - k * per), c > 1 ? ws + k : -1);
+    wt += n;
+    if (c > 1) {
+      split[wp++] = make_int4(u, ws, c, 0);
+      ws += c;
+    }
+  }
+}
+
+// dV = sum of a split unit's chunk partials and dK = scale * sum, in chunk
+// order, to bf16 (rows past the sequence are not written).
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_reduce_kernel(const BwdArgs a) {
+  const int nsplit = a.plan[1];
+  const int4* split = reinterpret_cast<const int4*>(a.plan) + 1 + a.plan_max_items;
+  const int nlevels = (a.N + 127) / 128;
+  const SeqSched sched{nullptr, a.nseq, a.N, a.Hkv, a.causal, nlevels, nullptr, 7};
+  constexpr int kPer = 128 * D / 4;  // float4 per [128][D] tensor
+  for (int sidx = blockIdx.x; sidx < nsplit; sidx += gridDim.x) {
+    const int4 sp = split[sidx];
+    const Unit un = decode_unit(sched, sp.x);
+    for (int e = threadIdx.x; e < 2 * kPer; e += blockDim.x) {
+      const int which = e / kPer, rem = e - which * kPer;
+      const int row = rem / (D / 4), c4 = rem - row * (D / 4);
+      const float4* src = reinterpret_cast<const float4*>(a.partials) + (static_cast<size_t>(sp.y) * 2 + which) * kPer + rem;
+      float4 acc = src[0];
+      for (int k = 1; k < sp.z; ++k) {
+        const float4 x = src[static_cast<size_t>(k) * 2 * kPer];
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+      }
+      const float mul = which == 0 ? 1.f : a.scale;
+      const int key = un.qb2 * 128 + row;
+      if (key < un.n) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which == 0 ? a.dv : a.dk) +
+                             (static_cast<size_t>(un.tok0 + key) * a.Hkv + un.h) * D + c4 * 4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x * mul, acc.y * mul), pack_bf16x2(acc.z * mul, acc.w * mul));
+      }
+    }
   }
 }
 

@@ -179,10 +179,28 @@ __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
 __device__ __forceinline__ bool kv_block_on(const FwdArgs& a, int h, int qb, int j) {
   return qb < a.nqb && __ldg(a.block_mask + (static_cast<size_t>(h) * a.nqb + qb) * a.nqb + j) != 0;
 }
+// Bit e set when key block base + e (< jend) is seen by query block qb0 or
+// qb0 + 1: eight independent loads per round, one round trip for eight
+// blocks (the mask is read through L2).
+__device__ __forceinline__ uint32_t kv_blocks_on8(const FwdArgs& a, int h, int qb0, int base, int jend) {
+  const uint8_t* r0 = a.block_mask + (static_cast<size_t>(h) * a.nqb + qb0) * a.nqb;
+  const bool has1 = qb0 + 1 < a.nqb;
+  uint32_t on = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int jj = base + e;
+    const uint8_t x0 = jj < jend ? __ldg(r0 + jj) : 0;
+    const uint8_t x1 = jj < jend && has1 ? __ldg(r0 + a.nqb + jj) : 0;
+    on |= (x0 | x1) ? (1u << e) : 0u;
+  }
+  return on;
+}
 __device__ __forceinline__ int next_kv_block(const FwdArgs& a, int h, int qb0, int j, int jend) {
   if (a.block_mask == nullptr) return j + 1;
-  for (int jj = j + 1; jj < jend; ++jj)
-    if (kv_block_on(a, h, qb0, jj) || kv_block_on(a, h, qb0 + 1, jj)) return jj;
+  for (int base = j + 1; base < jend; base += 8) {
+    const uint32_t on = kv_blocks_on8(a, h, qb0, base, jend);
+    if (on) return base + __ffs(on) - 1;
+  }
   return jend;
 }
 __device__ __forceinline__ int first_kv_block(const FwdArgs& a, int h, int qb0, int jend) {
@@ -192,7 +210,7 @@ __device__ __forceinline__ int first_kv_block(const FwdArgs& a, int h, int qb0, 
 __device__ __forceinline__ int count_kv_blocks(const FwdArgs& a, int h, int qb0, int jend) {
   if (a.block_mask == nullptr) return jend;
   int n = 0;
-  for (int j = next_kv_block(a, h, qb0, -1, jend); j < jend; j = next_kv_block(a, h, qb0, j, jend)) ++n;
+  for (int base = 0; base < jend; base += 8) n += __popc(kv_blocks_on8(a, h, qb0, base, jend));
   return n > 0 ? n : 1;
 }
 

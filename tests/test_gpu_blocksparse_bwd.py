@@ -112,3 +112,28 @@ def test_null_mask_is_an_error(fa):
     with pytest.raises(fa.FAError) as e:
         fa.fa_bwd_blocksparse(q, q, q, None, q, lse, q, *g, ws, ws.numel(), 1, 1, 1, 128, 64, 0, 0.125)
     assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_heavy_key_block_split_matches_oracle(fa, causal):
+    """A key block every query block sees (sliding window + global first
+    block): its dK/dV units are far longer than the rest and are split into
+    chunks whose partial sums are added afterwards; the result must match the
+    oracle and be bitwise reproducible."""
+    B, N, Hq, Hkv, d = 1, 4096, 4, 2, 128
+    q, k, v, do = synth.qkv_bf16(77 + int(causal), B, N, Hq, Hkv, d, with_dout=True)
+    nb = N // 128
+    mask = np.zeros((Hq, nb, nb), dtype=np.uint8)
+    for i in range(nb):
+        mask[:, i, max(0, i - 3):i + 1] = 1
+        mask[:, i, 0] = 1
+        if not causal:
+            mask[:, i, i:min(nb, i + 4)] = 1
+    got = _run(fa, q, k, v, do, mask, causal)
+    again = _run(fa, q, k, v, do, mask, causal)
+    for g, h in zip(got, again):
+        assert np.array_equal(g, h)
+    want = oracle.attn_bwd_blocksparse(q, k, v, do, mask, causal, 1 / math.sqrt(d))
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        rr = oracle.rel_rms(g, w)
+        assert rr <= G_REL_RMS, f"{name} rel-RMS {rr}"
