@@ -208,8 +208,8 @@ size_t vec_bytes(int tokens, int nseq, int Hq) {
 // sums follow the two workspace vectors. units = B * Hkv * ceil(N/128);
 // partial slots: 4 per SM (the plan leaves units unsplit beyond that).
 struct SparsePlanLayout {
-  long long units, max_slots, max_items, max_steps;
-  size_t plan_off, nbuf_off, sbase_off, steps_off, part_off, total;
+  long long units, max_slots, max_items, max_steps, rows;
+  size_t plan_off, nbuf_off, sbase_off, steps_off, rows_n_off, rows_base_off, rows_list_off, part_off, total;
 };
 SparsePlanLayout sparse_plan_layout(size_t base, int B, int Hq, int Hkv, int N, int d, int sms) {
   SparsePlanLayout L{};
@@ -223,7 +223,12 @@ SparsePlanLayout sparse_plan_layout(size_t base, int B, int Hq, int Hkv, int N, 
   L.nbuf_off = (L.plan_off + plan_ints * sizeof(int) + 255) & ~size_t(255);
   L.sbase_off = (L.nbuf_off + static_cast<size_t>(L.units) * sizeof(int) + 255) & ~size_t(255);
   L.steps_off = (L.sbase_off + static_cast<size_t>(L.units) * sizeof(int) + 255) & ~size_t(255);
-  L.part_off = (L.steps_off + static_cast<size_t>(L.max_steps) * sizeof(int) + 255) & ~size_t(255);
+  // dQ rows: per (query head, query tile) the visible key blocks
+  L.rows = static_cast<long long>(Hq) * nqb;
+  L.rows_n_off = (L.steps_off + static_cast<size_t>(L.max_steps) * sizeof(int) + 255) & ~size_t(255);
+  L.rows_base_off = (L.rows_n_off + static_cast<size_t>(L.rows) * sizeof(int) + 255) & ~size_t(255);
+  L.rows_list_off = (L.rows_base_off + static_cast<size_t>(L.rows) * sizeof(int) + 255) & ~size_t(255);
+  L.part_off = (L.rows_list_off + static_cast<size_t>(L.rows) * nqb * sizeof(int) + 255) & ~size_t(255);
   L.total = L.part_off + static_cast<size_t>(L.max_slots) * 2 * 128 * d * sizeof(float);
   return L;
 }
@@ -298,6 +303,18 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   fa::BwdArgs aq = a;
   aq.num_units = static_cast<int>(units_dq);
   const int g2 = static_cast<int>(units_dq < ds->sms ? units_dq : ds->sms);
+  // dQ on stream `st`; block-sparse: the rows' key-block lists before it
+  auto run_dq = [&](cudaStream_t st) -> bool {
+    if (SPARSE) {
+      const int rows = a.Hq * a.nqb;
+      fa::fa_bwd_rows_count_kernel<<<(rows + 7) / 8, 256, 0, st>>>(a, rows);
+      fa::fa_bwd_rows_scan_kernel<<<1, fa::kPlanThreads, 0, st>>>(a, rows);
+      fa::fa_bwd_rows_list_kernel<<<(rows + 7) / 8, 256, 0, st>>>(a, rows);
+      if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    kdq<<<g2, fa::kThreadsBwd, smem_dq, st>>>(tq, tk, tv, tdo, aq);
+    return cudaGetLastError() == cudaSuccess;
+  };
   if ((parts & FA_BWD_DKDV) && (parts & FA_BWD_DQ) && g1 > 0 && g2 > 0) {
     // dK/dV on the caller's stream and dQ on the side stream, both after the
     // preparation: their persistent CTAs have uneven causal work, and dQ's
@@ -313,8 +330,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
     if (cudaEventRecord(ds->fork, stream) != cudaSuccess || cudaStreamWaitEvent(ds->side, ds->fork, 0) != cudaSuccess)
       return FA_ERR_CUDA;
     if (!run_dkdv()) return FA_ERR_CUDA;
-    kdq<<<g2, fa::kThreadsBwd, smem_dq, ds->side>>>(tq, tk, tv, tdo, aq);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (!run_dq(ds->side)) return FA_ERR_CUDA;
     if (cudaEventRecord(ds->join, ds->side) != cudaSuccess || cudaStreamWaitEvent(stream, ds->join, 0) != cudaSuccess)
       return FA_ERR_CUDA;
     return FA_OK;
@@ -323,8 +339,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
     if (g1 > 0 && !run_dkdv()) return FA_ERR_CUDA;
   }
   if (parts & FA_BWD_DQ) {
-    if (g2 > 0) kdq<<<g2, fa::kThreadsBwd, smem_dq, stream>>>(tq, tk, tv, tdo, aq);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (g2 > 0 && !run_dq(stream)) return FA_ERR_CUDA;
   }
   return FA_OK;
 }
@@ -347,7 +362,8 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
   if (block_mask != nullptr) {
     L = sparse_plan_layout(2 * vb, nseq, Hq, Hkv, N, d, ds->sms);
     if (ws_bytes < L.total) return FA_ERR_WORKSPACE;
-    if (L.max_items > INT32_MAX / 4 || L.max_steps > INT32_MAX) return FA_ERR_UNSUPPORTED;
+    if (L.max_items > INT32_MAX / 4 || L.max_steps > INT32_MAX || L.rows * ((N + 127) / 128) > INT32_MAX)
+      return FA_ERR_UNSUPPORTED;
   }
   fa::BwdArgs a{};
   a.o = o;
@@ -393,6 +409,9 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
     a.plan_nbuf = reinterpret_cast<int*>(w + L.nbuf_off);
     a.plan_sbase = reinterpret_cast<int*>(w + L.sbase_off);
     a.plan_steps = reinterpret_cast<int*>(w + L.steps_off);
+    a.rows_n = reinterpret_cast<int*>(w + L.rows_n_off);
+    a.rows_base = reinterpret_cast<int*>(w + L.rows_base_off);
+    a.rows_list = reinterpret_cast<int*>(w + L.rows_list_off);
     a.partials = reinterpret_cast<float*>(w + L.part_off);
     a.plan_max_items = static_cast<int>(L.max_items);
     a.plan_max_slots = static_cast<int>(L.max_slots);

@@ -67,6 +67,11 @@ struct BwdArgs {
   int* plan_nbuf;   // visible steps per unit
   int* plan_sbase;  // first entry of each unit's steps in plan_steps
   int* plan_steps;  // every unit's visible steps, in order (unit after unit)
+  // block-sparse dQ: per row r = h * nqb + query tile, the visible key
+  // blocks (causal: at or below the diagonal) in order at rows_list[rows_base[r]..]
+  int* rows_n;
+  int* rows_base;
+  int* rows_list;
 };
 
 // ------------------------------------------------------------------ pre
@@ -87,31 +92,6 @@ __device__ __forceinline__ int ws_offset(int tok0, int seq) { return ((tok0 + 3)
 // runs the same pipeline.
 __device__ __forceinline__ bool bwd_block_on(const BwdArgs& a, int hq, int qb, int kb) {
   return __ldg(a.block_mask + (static_cast<size_t>(hq) * a.nqb + qb) * a.nqb + kb) != 0;
-}
-// Bit e set when key block base + e (< jend) is seen by query tile qt of
-// head h: eight independent loads per round (one round trip for eight).
-__device__ __forceinline__ uint32_t dq_blocks_on8(const BwdArgs& a, int h, int qt, int base, int jend) {
-  const uint8_t* r = a.block_mask + (static_cast<size_t>(h) * a.nqb + qt) * a.nqb;
-  uint32_t on = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) on |= (base + e < jend && __ldg(r + base + e) != 0) ? (1u << e) : 0u;
-  return on;
-}
-__device__ __forceinline__ int dq_next_block(const BwdArgs& a, int h, int qt, int j, int jend) {
-  for (int base = j + 1; base < jend; base += 8) {
-    const uint32_t on = dq_blocks_on8(a, h, qt, base, jend);
-    if (on) return base + __ffs(on) - 1;
-  }
-  return jend;
-}
-__device__ __forceinline__ int dq_first_block(const BwdArgs& a, int h, int qt, int jend) {
-  const int j = dq_next_block(a, h, qt, -1, jend);
-  return j < jend ? j : 0;
-}
-__device__ __forceinline__ int dq_count_blocks(const BwdArgs& a, int h, int qt, int jend) {
-  int n = 0;
-  for (int base = 0; base < jend; base += 8) n += __popc(dq_blocks_on8(a, h, qt, base, jend));
-  return n > 0 ? n : 1;
 }
 // Workspace entry r = (head h, index i) -> the token it holds, or -1 for a
 // gap / trailing filler entry: the last sequence whose block starts at or
@@ -286,6 +266,23 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const volatile int* abort = &sm.abort;
   const int group = args.Hq / args.Hkv;
   uint32_t prod_issued = 0, q_issued = 0;
+  // block-sparse: the unit's row of key blocks (count, first list entry);
+  // a row that sees nothing still visits block 0, every score masked
+  auto row_of = [&](const Unit& un, int& rn, int& rb) {
+    rn = 0;
+    rb = 0;
+    if constexpr (SPARSE) {
+      const int r = un.h * args.nqb + un.qb2;
+      rn = __ldg(args.rows_n + r);
+      rb = __ldg(args.rows_base + r);
+    }
+  };
+  auto block_at = [&](int rn, int rb, int j) -> int {
+    if constexpr (SPARSE)
+      return rn > 0 ? __ldg(args.rows_list + rb + j) : 0;
+    else
+      return j;
+  };
 
   if (warp == 8) {
     if (lane == 0) {
@@ -296,7 +293,9 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
         const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
-        const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
+        int rn, rb;
+        row_of(un, rn, rb);
+        const int nblk = SPARSE ? max(rn, 1) : jend;  // blocks visited
         const int hkv = un.h / group;
         if (!mbar_wait(smem_u32(&sm.q_empty), (it & 1) ^ 1, abort, args.timeout_ns)) {
           report_error(args.status, kStatusTimeout, 30);
@@ -309,8 +308,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         load_tile<D>(smem_u32(sm.q), &tm_q, qbar, un.h, row0);
         load_tile<D>(smem_u32(sm.dout), &tm_do, qbar, un.h, row0);
         q_issued = it + 1;
-        int jb = SPARSE ? dq_first_block(args, un.h, un.qb2, jend) : 0;  // key block of the j-th visit
-        for (int j = 0; j < nblk && ok; ++j, jb = SPARSE ? dq_next_block(args, un.h, un.qb2, jb, jend) : jb + 1) {
+        for (int j = 0; j < nblk && ok; ++j) {
+          const int jb = block_at(rn, rb, j);  // key block of the j-th visit
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = kv_prod % STAGES;
             if (!mbar_wait(smem_u32(&sm.kv_empty[slot]), ((kv_prod / STAGES) & 1) ^ 1, abort, args.timeout_ns)) {
@@ -346,7 +345,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         if (u >= num_units) break;
         const Unit un = decode_unit(sched, u);
         const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
-        const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
+        int rn, rb;
+        row_of(un, rn, rb);
+        const int nblk = SPARSE ? max(rn, 1) : jend;  // blocks visited
+        (void)rb;
         if (!(ok = wait(&sm.q_full, it & 1, 40))) break;
         const uint32_t qa = smem_u32(sm.q), doa = smem_u32(sm.dout);
         // prologue: S(0)
@@ -401,15 +403,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
       const int jend = args.causal ? min((un.n + 127) / 128, un.qb2 + 1) : (un.n + 127) / 128;
-      const int nblk = SPARSE ? dq_count_blocks(args, un.h, un.qb2, jend) : jend;  // blocks visited
-      int jb = SPARSE ? dq_first_block(args, un.h, un.qb2, jend) : 0;  // key block of the j-th visit
+      int rn, rb;
+      row_of(un, rn, rb);
+      const int nblk = SPARSE ? max(rn, 1) : jend;  // blocks visited
       const int row = un.qb2 * kBM + r_in_tile;
       const bool valid = row < un.n;
       const size_t wi = static_cast<size_t>(un.h) * args.ws_stride + ws_offset(un.tok0, un.seq) + row;
       const float lse2 = valid ? args.lse2[wi] : INFINITY;
       const float dval = valid ? args.dvec[wi] : 0.f;
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;
-      for (int j = 0; j < nblk; ++j, jb = SPARSE ? dq_next_block(args, un.h, un.qb2, jb, jend) : jb + 1) {
+      for (int j = 0; j < nblk; ++j) {
+        const int jb = block_at(rn, rb, j);  // key block of the j-th visit
         const int sb = j & 1;
         const uint32_t par = sb ? (sc1 & 1) : (sc0 & 1);
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[sb]), par, abort, args.timeout_ns));
@@ -424,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         float p[64];
         const int c0 = jb * kBN + half * 64;
         // block-sparse: a visit of a block this tile may not see (a unit that sees none)
-        const bool off = SPARSE && !bwd_block_on(args, un.h, un.qb2, jb);
+        const bool off = SPARSE && rn == 0;
         const bool masked_blk = off || __any_sync(0xffffffffu, c0 + 63 > limit);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -1052,6 +1056,62 @@ __global__ void __launch_bounds__(256) fa_bwd_reduce_kernel(const BwdArgs a) {
         *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x * mul, acc.y * mul), pack_bf16x2(acc.z * mul, acc.w * mul));
       }
     }
+  }
+}
+
+// ------------------------------------------------------------------ block-sparse dQ rows
+// The key blocks each (query head, query tile) row sees, as lists: counted
+// (one warp per row, 32 mask bytes at a time), prefix-summed (one CTA), then
+// written in order (ballot ranks). The dQ kernel reads block j of its row.
+__device__ __forceinline__ int dq_row_end(const BwdArgs& a, int qt) { return a.causal ? min(a.nqb, qt + 1) : a.nqb; }
+
+__global__ void __launch_bounds__(256) fa_bwd_rows_count_kernel(const BwdArgs a, int rows) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= rows) return;  // uniform over the warp
+  const int qt = r % a.nqb, jend = dq_row_end(a, qt);
+  const uint8_t* m = a.block_mask + static_cast<size_t>(r) * a.nqb;
+  int n = 0;
+  for (int base = 0; base < jend; base += 32)
+    n += __popc(__ballot_sync(0xffffffffu, base + lane < jend && __ldg(m + base + lane) != 0));
+  if (lane == 0) a.rows_n[r] = n;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) fa_bwd_rows_scan_kernel(const BwdArgs a, int rows) {
+  __shared__ int part[kPlanThreads];
+  const int tid = threadIdx.x;
+  const int seg = (rows + kPlanThreads - 1) / kPlanThreads;
+  const int r0 = min(rows, tid * seg), r1 = min(rows, r0 + seg);
+  int sum = 0;
+  for (int r = r0; r < r1; ++r) sum += a.rows_n[r];
+  part[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int i = 0; i < kPlanThreads; ++i) {
+      const int x = part[i];
+      part[i] = acc;
+      acc += x;
+    }
+  }
+  __syncthreads();
+  int acc = part[tid];
+  for (int r = r0; r < r1; ++r) {
+    a.rows_base[r] = acc;
+    acc += a.rows_n[r];
+  }
+}
+
+__global__ void __launch_bounds__(256) fa_bwd_rows_list_kernel(const BwdArgs a, int rows) {
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= rows) return;  // uniform over the warp
+  const int qt = r % a.nqb, jend = dq_row_end(a, qt);
+  const uint8_t* m = a.block_mask + static_cast<size_t>(r) * a.nqb;
+  int pos = a.rows_base[r];
+  for (int base = 0; base < jend; base += 32) {
+    const bool on = base + lane < jend && __ldg(m + base + lane) != 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, on);
+    if (on) a.rows_list[pos + __popc(bal & ((1u << lane) - 1u))] = base + lane;
+    pos += __popc(bal);
   }
 }
 
