@@ -137,3 +137,47 @@ def test_heavy_key_block_split_matches_oracle(fa, causal):
     for name, g, w in zip(("dq", "dk", "dv"), got, want):
         rr = oracle.rel_rms(g, w)
         assert rr <= G_REL_RMS, f"{name} rel-RMS {rr}"
+
+
+def test_split_units_gqa_d64_with_unseen_key_blocks(fa):
+    """GQA group 4, d = 64, two global key columns (split units) beside key
+    blocks nothing sees (forced zero visits): matches the oracle, the unseen
+    blocks' dK/dV rows are exactly 0, bitwise reproducible."""
+    B, N, Hq, Hkv, d = 2, 3000, 8, 2, 64
+    q, k, v, do = synth.qkv_bf16(91, B, N, Hq, Hkv, d, with_dout=True)
+    nb = (N + 127) // 128
+    mask = np.zeros((Hq, nb, nb), dtype=np.uint8)
+    for i in range(nb):
+        mask[:, i, max(0, i - 1):i + 1] = 1
+        mask[:, i, 0] = 1
+        mask[:, i, 5] = 1
+    mask[:, :, 9] = 0   # key block 9: seen by nothing
+    mask[:, :, 12] = 0
+    got = _run(fa, q, k, v, do, mask, True)
+    again = _run(fa, q, k, v, do, mask, True)
+    for g, h in zip(got, again):
+        assert np.array_equal(g, h)
+    _, k_zero = _zero_rows(mask, N, Hq, Hkv, True)
+    assert k_zero[9 * 128:10 * 128].all()
+    dq, dk, dv = got
+    assert np.all(dk.transpose(0, 2, 1, 3)[:, k_zero.T] == 0)
+    assert np.all(dv.transpose(0, 2, 1, 3)[:, k_zero.T] == 0)
+    want = oracle.attn_bwd_blocksparse(q, k, v, do, mask, True, 1 / math.sqrt(d))
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        rr = oracle.rel_rms(g, w)
+        assert rr <= G_REL_RMS, f"{name} rel-RMS {rr}"
+
+
+def test_workspace_too_small_is_an_error(fa):
+    B, N, Hq, Hkv, d = 1, 512, 2, 1, 64
+    q = torch.zeros((B, N, Hq, d), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((B, N, Hkv, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((B, Hq, N), dtype=torch.float32, device="cuda")
+    mask = torch.ones((Hq, 4, 4), dtype=torch.uint8, device="cuda")
+    need = fa.fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d)
+    assert need > fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    g = [torch.empty_like(q), torch.empty_like(kv), torch.empty_like(kv)]
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_bwd_blocksparse(q, kv, kv, mask, q, lse, q, *g, ws, ws.numel(), B, Hq, Hkv, N, d, 0, 0.125)
+    assert e.value.status == fa.FA_ERR_WORKSPACE
