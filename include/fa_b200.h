@@ -212,7 +212,8 @@ int fa_fwd_kvcache_num_splits(int B, int Hkv, int Ncache, int d);
  *              sequence of the batch; with causal = 1 the causal mask applies
  *              too.
  * Only visited key blocks are loaded and multiplied. A query row that sees no
- * key gets O = 0 and LSE = -inf. NULL mask: FA_ERR_INVALID_ARG.
+ * key gets O = 0 and LSE = -inf. NULL mask: FA_ERR_INVALID_ARG; N > 131072:
+ * FA_ERR_UNSUPPORTED.
  */
 fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask, void* o,
                                float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale,

@@ -521,6 +521,7 @@ fa_status_t fa_fwd_blocksparse(const void* q, const void* k, const void* v, cons
   if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
   if (B == 0 || N == 0) return FA_OK;
   if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (N > 131072) return FA_ERR_UNSUPPORTED;  // the softmax warps hold a mask row in 32 x 32 bits
   return fwd_dispatch(q, k, v, o, lse, nullptr, B, N, B * N, Hq, Hkv, d, causal, scale, stream, block_mask);
 }
 

@@ -214,6 +214,49 @@ __device__ __forceinline__ int count_kv_blocks(const FwdArgs& a, int h, int qb0,
   return n > 0 ? n : 1;
 }
 
+// The softmax warps' copy of a unit's two mask rows: lane i holds, in bit e
+// of rows[t], whether query block qb0 + t sees key block 32 i + e (< jend).
+// Loaded once per unit (64 independent byte loads per lane, one round trip);
+// the walk over visible blocks and the per-tile flags are then warp
+// operations on registers. nqb <= 1024 (32 blocks per lane).
+struct WarpMaskRows {
+  uint32_t rows[2];
+};
+__device__ __forceinline__ WarpMaskRows warp_mask_rows(const FwdArgs& a, int h, int qb0, int jend, int lane) {
+  WarpMaskRows w{{0u, 0u}};
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (qb0 + t >= a.nqb) continue;
+    const uint8_t* r = a.block_mask + (static_cast<size_t>(h) * a.nqb + qb0 + t) * a.nqb;
+    uint8_t x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = lane * 32 + e < jend ? __ldg(r + lane * 32 + e) : 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) w.rows[t] |= x[e] ? (1u << e) : 0u;
+  }
+  return w;
+}
+// First visible block (either tile) after j, or jend; warp-uniform.
+__device__ __forceinline__ int warp_next_block(const WarpMaskRows& w, int j, int jend, int lane) {
+  const int from = j + 1;
+  uint32_t word = w.rows[0] | w.rows[1];
+  if (lane * 32 + 31 < from)
+    word = 0;
+  else if (lane * 32 < from)
+    word &= ~((1u << (from - lane * 32)) - 1u);
+  const uint32_t bal = __ballot_sync(0xffffffffu, word != 0);
+  if (bal == 0) return jend;
+  const int src = __ffs(bal) - 1;
+  const uint32_t ws = __shfl_sync(0xffffffffu, word, src);
+  return src * 32 + __ffs(ws) - 1;
+}
+__device__ __forceinline__ int warp_count_blocks(const WarpMaskRows& w) {
+  return __reduce_add_sync(0xffffffffu, __popc(w.rows[0] | w.rows[1]));
+}
+__device__ __forceinline__ bool warp_tile_on(const WarpMaskRows& w, int tile, int jb) {
+  return (__shfl_sync(0xffffffffu, w.rows[tile], jb >> 5) >> (jb & 31)) & 1u;
+}
+
 // Exponentials of 2*NP consecutive columns of one row: p = 2^(s*cj - m),
 // packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[NP] for
 // the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs;
@@ -505,7 +548,10 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       if (u >= num_units) break;
       const Unit un = decode_unit(sched, u);
       const int jend = num_kv_blocks(un, args.causal);
-      const int nblk = SPARSE ? count_kv_blocks(args, un.h, un.qb2 * 2, jend) : jend;  // key blocks visited
+      WarpMaskRows wm{{0u, 0u}};
+      if constexpr (SPARSE) wm = warp_mask_rows(args, un.h, un.qb2 * 2, jend, lane);
+      int nblk = jend;  // key blocks visited (block-sparse: at least one, block 0 fully masked)
+      if constexpr (SPARSE) nblk = max(warp_count_blocks(wm), 1);
       const int row = un.qb2 * 2 * kBM + tile * kBM + r_in_tile;  // row within the sequence
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;  // last visible key
       // scores are kept in base-2 units t = s * cj; cj = scale*log2(e) for
@@ -521,8 +567,12 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         sv_max = fmaxf(sv_max, 1e-30f);
       }
       float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
-      int jb = SPARSE ? first_kv_block(args, un.h, un.qb2 * 2, jend) : 0;  // key block of the j-th visit
-      for (int j = 0; j < nblk; ++j, jb = SPARSE ? next_kv_block(args, un.h, un.qb2 * 2, jb, jend) : jb + 1) {
+      int jb = 0;  // key block of the j-th visit
+      if constexpr (SPARSE) {
+        jb = warp_next_block(wm, -1, jend, lane);
+        if (jb >= jend) jb = 0;
+      }
+      for (int j = 0; j < nblk; ++j, jb = SPARSE ? warp_next_block(wm, jb, jend, lane) : jb + 1) {
         float cj = cl, pmul = 1.f;
         if constexpr (F8) {
           cj = cl * sq * args.k_scale[kvs + jb];
@@ -536,7 +586,7 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
         ++sc;
         const int kv0 = jb * kBN + 64 * half;  // first key of this half
         // block-sparse: the whole block is hidden from this tile (uniform over the tile)
-        const bool tile_on = !SPARSE || kv_block_on(args, un.h, un.qb2 * 2 + tile, jb);
+        const bool tile_on = !SPARSE || warp_tile_on(wm, tile, jb);
         // warp-uniform: every lane of a warp takes the same masked/unmasked path
         const bool masked_blk = !tile_on || __any_sync(0xffffffffu, kv0 + 63 > limit);
         // pass 1: this half's row maximum, exchanged with the partner half
@@ -646,7 +696,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
       if (valid && half == 0) {
         const size_t li = varlen ? (static_cast<size_t>(un.h) * args.lse_head_stride + un.tok0 + row)
                                  : (static_cast<size_t>(un.seq * args.Hq + un.h) * args.lse_head_stride + row);
-        args.lse[li] = !SPARSE || lt > 0.f ? m * 0.6931471805599453f + logf(lt) : -INFINITY;
+        // one explicit fused multiply-add: every instantiation rounds the LSE alike
+        args.lse[li] = !SPARSE || lt > 0.f ? __fmaf_rn(m, 0.6931471805599453f, logf(lt)) : -INFINITY;
       }
     }
     if (!ok) sm.abort = 1;
