@@ -104,17 +104,26 @@ def kernel_source_hash(kernel):
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel):
+def traffic_for(kernel, shape):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
-    when the kernel's device sources changed since those counters were taken."""
+    when the kernel's device sources changed since those counters were taken
+    or the capture ran another shape than `shape`."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p) or kernel not in KERNEL_HEADER:
         return None
     j = json.load(open(p))
     e = j.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash(kernel):
+    if not e or e.get("source_hash") != kernel_source_hash(kernel) or e.get("shape") != shape:
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def step_shape(B, Hq, Hkv, N, d, causal):
+    return f"B={B} Hq={Hq} Hkv={Hkv} N={N} d={d} causal={int(bool(causal))}"
+
+
+def decode_shape_key(B, Nq, Hq, Hkv, Nc, d):
+    return f"B={B} Nq={Nq} Hq={Hq} Hkv={Hkv} Ncache={Nc} d={d}"
 
 
 class ClockSampler:
@@ -353,12 +362,12 @@ def run_ours(args):
     if dom["bound"] == "tensor":
         roofline = {"bound": "tensor", "kernel": dom["kernel"], "achieved": dom["achieved_tflops"],
                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": dom["frac"],
-                    "traffic": traffic_for(dom["kernel"]),
+                    "traffic": traffic_for(dom["kernel"], step_shape(B, Hq, Hkv, N, d, causal)),
                     "peak_source": f"{pk['source']} bf16 burst (cuBLAS)", "kernels": kernels}
     else:
         roofline = {"bound": "hbm", "kernel": dom["kernel"], "achieved": dom["achieved_gbs"],
                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dom["frac"],
-                    "traffic": traffic_for(dom["kernel"]), "peak_source": f"{pk['source']} HBM copy",
+                    "traffic": traffic_for(dom["kernel"], step_shape(B, Hq, Hkv, N, d, causal)), "peak_source": f"{pk['source']} HBM copy",
                     "kernels": kernels}
 
     # end to end through the public API with host buffers (pinned), copies timed
@@ -552,7 +561,7 @@ def run_decode(args):
     per_kernel = byts / (ms_per_step * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "fa_decode_kernel" + (" + fa_decode_merge_kernel" if splits > 1 else ""),
                 "achieved": per_kernel, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": per_kernel / pk["hbm_gbs"],
-                "traffic": traffic_for("fa_decode_kernel"), "peak_source": f"{pk['source']} HBM copy",
+                "traffic": traffic_for("fa_decode_kernel", decode_shape_key(B, Nq, Hq, Hkv, Nc, d)), "peak_source": f"{pk['source']} HBM copy",
                 "bytes_per_launch": byts, "num_splits": splits}
     e2e = None
     if args.e2e_steps > 0:

@@ -22,7 +22,7 @@
 // rows (lanes) 32*(w%4).. and the column half w/4 of each 128-column tile.
 #pragma once
 
-#include "fa_fwd_kernel.cuh"
+#include "fa_tile.cuh"
 
 namespace fa {
 

@@ -76,3 +76,17 @@ def test_null_mask_is_an_error(fa):
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd_blocksparse(q, q, q, None, o, lse, 1, 1, 1, 128, 64, 0, 0.125)
     assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+def test_too_many_key_blocks_is_unsupported(fa):
+    """The forward holds one query block's mask row in its warp's registers
+    (32 key blocks per lane): N above 1024 key blocks is refused up front."""
+    N = 131072 + 1
+    q = torch.zeros((1, N, 1, 64), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 1, N), dtype=torch.float32, device="cuda")
+    nb = (N + 127) // 128
+    mask = torch.ones((1, nb, nb), dtype=torch.uint8, device="cuda")
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_fwd_blocksparse(q, q, q, mask, o, lse, 1, 1, 1, N, 64, 0, 0.125)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
