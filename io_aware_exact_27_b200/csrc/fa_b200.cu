@@ -242,12 +242,15 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES, SPARSE>;
   const int smem_dq = static_cast<int>(sizeof(fa::DqSmem<D, STAGES>)) + 1024;
   const int smem_dkv = static_cast<int>(sizeof(fa::DkvSmem<D, STAGES>)) + 1024;
+  auto kpre = fa::fa_bwd_pre_kernel<D>;
+  const int smem_pre = static_cast<int>(sizeof(fa::PreSmem)) + 128;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     bool& done = ds->bwd_attr[D == 128 ? 1 : 0][SPARSE ? 1 : 0];
     if (!done) {
       if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess ||
-          cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv) != cudaSuccess)
+          cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv) != cudaSuccess ||
+          cudaFuncSetAttribute(kpre, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pre) != cudaSuccess)
         return FA_ERR_CUDA;
       done = true;
     }
@@ -261,14 +264,15 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   if ((st = encode_rows(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hq, D)) != FA_OK) return st;
   a.timeout_ns = g_timeout_ns.load();
   a.status = ds->status;
-  // D and LSE in base 2: 8 warps per block, each warp kPrePasses x 32/(D/8)
-  // entries per pass; at most 8 resident blocks per SM
-  const long long rows = static_cast<long long>(a.Hq) * a.ws_stride;
-  const long long per_block = 8LL * (32 / (D / 8)) * fa::kPrePasses;
-  long long pre_blocks = (rows + per_block - 1) / per_block;
-  if (pre_blocks > static_cast<long long>(ds->sms) * 8) pre_blocks = static_cast<long long>(ds->sms) * 8;
+  // D and LSE in base 2: one CTA per SM (a ring of 3 x 64 KB of O and dO
+  // chunks), at most one per chunk
+  const long long entries = static_cast<long long>(a.Hq) * a.total_T;
+  const long long chunk_entries = fa::kPreChunk / (D * 2);
+  long long pre_blocks = (entries + chunk_entries - 1) / chunk_entries;
+  if (pre_blocks > ds->sms) pre_blocks = ds->sms;
+  if (pre_blocks < 1) pre_blocks = 1;
   if (parts & FA_BWD_PREPARE) {
-    fa::fa_bwd_pre_kernel<D><<<static_cast<int>(pre_blocks), 256, 0, stream>>>(a);
+    kpre<<<static_cast<int>(pre_blocks), fa::kPreThreads, smem_pre, stream>>>(a);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   fa::BwdArgs akv = a;
