@@ -11,6 +11,7 @@
 
 #include "../../include/fa_b200.h"
 #include "fa_bwd_kernel.cuh"
+#include "fa_bwd_pre_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_decode_kernel.cuh"
 #include "fa_merge_kernel.cuh"
