@@ -52,10 +52,14 @@ def parse():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
-    ap.add_argument("--workload", default="attention", choices=["attention", "decode", "ring", "fp8", "blocksparse"],
+    ap.add_argument("--workload", default="attention",
+                    choices=["attention", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"],
                     help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
                          "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated); "
-                         "fp8: Hadamard-rotated e4m3 quantisation + fp8 forward (B=2 H=16 N=8192 d=128 causal)")
+                         "fp8: Hadamard-rotated e4m3 quantisation + fp8 forward (B=2 H=16 N=8192 d=128 causal); "
+                         "sweep: causal fwd+bwd at N = 2K..32K with B*N = 32K tokens (H=16 d=128), plus the tiny "
+                         "B=1 H=2 N=256 d=64 case; varlen: 24 packed causal sequences of U[128,4096] tokens, "
+                         "fwd+bwd (H=16 d=128)")
     ap.add_argument("--ring-shape", default="1,32,8,16384,128",
                     help="B,Hq,Hkv,N,d of the ring workload (causal; N split over the ring)")
     ap.add_argument("--ring-ranks", type=int, default=4, help="ranks emulated on one GPU (--gpus 1)")
@@ -184,13 +188,14 @@ def dist_setup(args):
 
 # ----------------------------------------------------------------- reference arm (CPU oracle)
 
-def oracle_sample(budget_s, with_bwd):
+def oracle_sample(budget_s, with_bwd, w=None):
     """Times the fp64 oracle on whole (batch, head) problems of the workload
-    until `budget_s` is spent; returns (TFLOP/s, heads done, seconds, cores)."""
+    (default: the bench's) until `budget_s` is spent; returns (TFLOP/s, heads
+    done, seconds, cores)."""
     import numpy as np
     import oracle
     import synth
-    w = WORKLOAD
+    w = w or WORKLOAD
     q, k, v, do = synth.qkv_bf16(0, w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], with_dout=True)
     scale = 1.0 / math.sqrt(w["d"])
     per_head = fwd_flops(1, 1, w["N"], w["d"], w["causal"]) * (3.5 if with_bwd else 1.0)
@@ -1326,8 +1331,326 @@ def run_bs_reference(args):
     return 0
 
 
+# ----------------------------------------------------------------- sweep over N
+
+SWEEP_TOKENS = 32768
+SWEEP_NS = (2048, 4096, 8192, 16384, 32768)
+SWEEP_H, SWEEP_D = 16, 128
+TINY = (1, 2, 2, 256, 64, False)  # B, Hq, Hkv, N, d, causal
+
+
+def sweep_workload(N):
+    return {"B": SWEEP_TOKENS // N, "Hq": SWEEP_H, "Hkv": SWEEP_H, "N": N, "d": SWEEP_D, "causal": True}
+
+
+def run_sweep(args):
+    """Causal fwd+bwd at every N of SWEEP_NS (B = 32K / N tokens, H=16,
+    d=128), each timed on its own (L2 flushed before every step), and the tiny
+    non-causal case (launch-bound: microseconds and GB/s). One step of the
+    line = one fwd+bwd at every N; the value is the flops of that step over
+    its time."""
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        budget = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+        vals = [oracle_sample(budget, True, sweep_workload(SWEEP_NS[0])) for _ in range(args.warmup + args.steps)]
+        vals = vals[args.warmup:]
+        tf = sum(v[0] for v in vals) / len(vals)
+        sample = f"{vals[0][1]} (batch, head) problems of the N=2048 point per step, fp64 numpy, fwd+bwd"
+        print(json.dumps({"metric": METRIC + " (sweep)", "value": tf, "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "impl": "reference",
+                          "config": {"workload": f"causal attention fwd+bwd sweep, N in {list(SWEEP_NS)}, "
+                                                 f"B*N = {SWEEP_TOKENS}, Hq=Hkv={SWEEP_H}, d={SWEEP_D}"},
+                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return 0
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    import synth
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk = peaks()
+
+    def time_point(B, Hq, Hkv, N, d, causal):
+        q, k, v, do = (t.to(dev) for t in synth.qkv_bf16(rank, B, N, Hq, Hkv, d, with_dout=True))
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        wsb = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        scale = 1.0 / math.sqrt(d)
+        fwd = lambda: fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), scale, sptr)
+        bwd = lambda: fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, wsb, B, Hq, Hkv, N, d, int(causal), scale, sptr)
+        for _ in range(args.warmup):
+            fwd()
+            bwd()
+        ms = []
+        for with_bwd in (False, True):
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                fwd()
+                if with_bwd:
+                    bwd()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps)
+        if fa.fa_get_status(sptr) != fa.FA_OK:
+            raise SystemExit(f"device status error at N={N}")
+        return ms[0], ms[1]
+
+    steps = max(3, min(args.steps, 20))
+    args.steps = steps
+    points, tot_flops, tot_ms = [], 0.0, 0.0
+    if pg:
+        pg.barrier()
+    with ClockSampler(local) as clk:
+        for N in SWEEP_NS:
+            w = sweep_workload(N)
+            f = fwd_flops(w["B"], w["Hq"], N, w["d"], True)
+            ms_f, ms_s = time_point(w["B"], w["Hq"], w["Hkv"], N, w["d"], True)
+            points.append({"N": N, "B": w["B"], "fwd_ms": ms_f, "step_ms": ms_s,
+                           "fwd_tflops": f / (ms_f * 1e-3) / 1e12,
+                           "bwd_tflops": 2.5 * f / ((ms_s - ms_f) * 1e-3) / 1e12,
+                           "step_tflops": 3.5 * f / (ms_s * 1e-3) / 1e12,
+                           "fwd_frac": f / (ms_f * 1e-3) / 1e12 / pk["bf16_tflops"]})
+            tot_flops += 3.5 * f
+            tot_ms += ms_s
+            torch.cuda.empty_cache()
+        B, Hq, Hkv, N, d, causal = TINY
+        ms_f, ms_s = time_point(B, Hq, Hkv, N, d, causal)
+    tiny_bytes = (2 * B * N * Hq * d + 2 * B * N * Hkv * d) * 2 + B * Hq * N * 4  # Q, K, V read; O, LSE written
+    tiny = {"B": B, "Hq": Hq, "N": N, "d": d, "causal": causal, "fwd_us": ms_f * 1e3, "step_us": ms_s * 1e3,
+            "fwd_gbs": tiny_bytes / (ms_f * 1e-3) / 1e9}
+    if pg:
+        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        tot_ms = float(t.item())
+    value = tot_flops * world / (tot_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, heads, el, cores = oracle_sample(args.cpu_budget_s, True, sweep_workload(SWEEP_NS[0]))
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{heads} (batch, head) problems of the N=2048 point, fp64 numpy, fwd+bwd, {el:.1f} s"}
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    p16 = next(p for p in points if p["N"] == 16384)
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel (N=16384 point)", "achieved": p16["fwd_tflops"],
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": p16["fwd_frac"], "traffic": None,
+                "peak_source": f"{pk['source']} bf16 burst (cuBLAS)"}
+    cfg = {"workload": f"bf16 causal attention fwd+bwd sweep, N in {list(SWEEP_NS)} at B*N = {SWEEP_TOKENS} "
+                       f"tokens, Hq=Hkv={SWEEP_H}, d={SWEEP_D}; plus B=1 H=2 N=256 d=64 non-causal",
+           "parallelism": f"dp{world}" if world > 1 else "single", "l2": "flushed before every step"}
+    line = {"metric": METRIC + " (sweep)", "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": None, "clocks": clocks,
+            "gpu_launches": 4 * steps * (len(SWEEP_NS) + 1) + steps * (len(SWEEP_NS) + 1),
+            "points": points, "tiny": tiny}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+
+# ----------------------------------------------------------------- varlen (packed sequences)
+
+VARLEN_H, VARLEN_D = 16, 128
+
+
+def varlen_flops(lengths, H, d):
+    return sum(4.0 * H * int(n) * int(n) * d / 2.0 for n in lengths)  # causal forward
+
+
+def varlen_oracle_sample(budget_s, lengths, cu):
+    """The fp64 oracle on whole (sequence, head) problems of the packed batch,
+    fwd+bwd, until `budget_s` is spent; returns (TFLOP/s, problems, seconds, cores)."""
+    import oracle
+    import synth
+    q, k, v, do, _ = synth.qkv_varlen_bf16(0, lengths, VARLEN_H, VARLEN_H, VARLEN_D, with_dout=True)
+    scale = 1.0 / math.sqrt(VARLEN_D)
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    while done < len(lengths) * VARLEN_H:
+        i, h = divmod(done, VARLEN_H)
+        a, b = int(cu[i]), int(cu[i + 1])
+        sl = (None, slice(a, b), slice(h, h + 1))
+        oracle.attn_fwd(q[sl], k[sl], v[sl], True, scale)
+        oracle.attn_bwd(q[sl], k[sl], v[sl], do[sl], True, scale)
+        flops += 3.5 * varlen_flops([b - a], 1, VARLEN_D)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    return flops / el / 1e12, done, el, os.cpu_count()
+
+
+def run_varlen(args):
+    """Packed causal fwd+bwd over 24 sequences of U[128, 4096] tokens (seeded:
+    T = 52,929), Hq = Hkv = 16, d = 128, through fa_fwd_varlen / fa_bwd_varlen;
+    L2 flushed before every step; the forward timed alone in a second pass."""
+    import synth
+    world, rank, local = dist_setup(args)
+    lengths = synth.varlen_lengths(rank)
+    cu_h = synth.cu_seqlens_of(lengths)
+    T, mx = int(cu_h[-1]), int(lengths.max())
+    f = varlen_flops(lengths, VARLEN_H, VARLEN_D)
+    wl = (f"bf16 causal varlen attention fwd+bwd, {len(lengths)} sequences of U[128,4096] tokens "
+          f"(T={T}), Hq=Hkv={VARLEN_H}, d={VARLEN_D}")
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        budget = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
+        vals = [varlen_oracle_sample(budget, lengths, cu_h) for _ in range(args.warmup + args.steps)][args.warmup:]
+        tf = sum(v[0] for v in vals) / len(vals)
+        print(json.dumps({"metric": METRIC + " (varlen)", "value": tf, "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "impl": "reference", "config": {"workload": wl},
+                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle",
+                                           "sample": f"{vals[0][1]} (sequence, head) problems per step, fp64 "
+                                                     f"numpy, fwd+bwd"},
+                          "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
+        return 0
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    import io_aware_exact_27_b200 as fa
+    H, d = VARLEN_H, VARLEN_D
+    q_h, k_h, v_h, do_h, _ = synth.qkv_varlen_bf16(rank, lengths, H, H, d, with_dout=True)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    cu = torch.from_numpy(cu_h).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nseq = len(lengths)
+    wsb = fa.fa_bwd_workspace_size(T, nseq, H, d)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+    scale = 1.0 / math.sqrt(d)
+    fwd = lambda: fa.fa_fwd_varlen(q, k, v, o, lse, cu, nseq, mx, T, H, H, d, 1, scale, sptr)
+    bwd = lambda: fa.fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, ws, wsb, cu, nseq, mx, T, H, H, d, 1, scale,
+                                   sptr)
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error during warm-up")
+    if pg:
+        pg.barrier()
+    ms = []
+    with ClockSampler(local) as clk:
+        for with_bwd in (True, False):
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record(stream)
+                fwd()
+                if with_bwd:
+                    bwd()
+                ev[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps)
+    if fa.fa_get_status(sptr) != fa.FA_OK:
+        raise SystemExit("device status error")
+    ms_s, ms_f = ms
+    if pg:
+        t = torch.tensor([ms_s, ms_f], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_s, ms_f = (float(x) for x in t.tolist())
+    value = 3.5 * f * world / (ms_s * 1e-3) / 1e12
+    pk = peaks()
+    fwd_tf = f / (ms_f * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel (varlen)", "achieved": fwd_tf,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_tf / pk["bf16_tflops"], "traffic": None,
+                "peak_source": f"{pk['source']} bf16 burst (cuBLAS)",
+                "backward_tflops": 2.5 * f / ((ms_s - ms_f) * 1e-3) / 1e12}
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+        outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for dst, src in zip((q, k, v, do), pin):
+                dst.copy_(src, non_blocking=True)
+            fwd()
+            bwd()
+            for dst, src in zip(outs, (o, lse, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": 3.5 * f * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)}
+    cpu = None
+    if rank == 0 and world == 1:
+        tf, n, el, cores = varlen_oracle_sample(args.cpu_budget_s, lengths, cu_h)
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} of {nseq * H} (sequence, head) problems, fp64 numpy, fwd+bwd, {el:.1f} s"}
+    clocks = clk.summary()
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = {"workload": wl, "T": T, "nseq": nseq, "Hq": H, "Hkv": H, "d": d, "causal": True,
+           "parallelism": f"dp{world}" if world > 1 else "single", "l2": "flushed before every step"}
+    line = {"metric": METRIC + " (varlen)", "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_s, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": 5 * args.steps,
+            "forward_ms": ms_f}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+
 def main():
     args = parse()
+    if args.workload == "sweep":
+        return run_sweep(args)
+    if args.workload == "varlen":
+        return run_varlen(args)
     if args.workload == "blocksparse":
         return run_blocksparse(args)
     if args.workload == "fp8":

@@ -1,0 +1,45 @@
+"""bench.py's JSON line, on the CPU: every workload's reference arm (the fp64
+oracle timed on the host) prints exactly one line with the contract's keys;
+the DRAM-traffic lookup only answers for the shape it was captured on."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+             "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
+
+
+@pytest.mark.parametrize("workload", ["attention", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"])
+def test_reference_arm_prints_one_contract_line(workload):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          workload, "--steps", "1", "--warmup", "0", "--cpu-budget-s", "0.3"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert BASE_KEYS <= set(j), BASE_KEYS - set(j)
+    assert j["impl"] == "reference" and j["n_gpus"] == 1 and j["steps"] == 1
+    assert j["value"] > 0 and j["cpu_baseline"]["value"] == j["value"]
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
+    assert isinstance(j["config"]["workload"], str) and j["config"]["workload"]
+
+
+def test_traffic_lookup_is_keyed_by_shape():
+    import bench
+    j = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    for kernel, e in j.items():
+        if kernel.startswith("_"):
+            continue
+        assert isinstance(e["shape"], str) and e["dram_bytes_per_launch"] > 0
+        if e["source_hash"] == bench.kernel_source_hash(kernel):
+            assert bench.traffic_for(kernel, e["shape"]) == e["dram_bytes_per_launch"]
+        assert bench.traffic_for(kernel, e["shape"] + " other") is None
