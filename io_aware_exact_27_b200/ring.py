@@ -28,7 +28,10 @@ dK/dV accumulators of a shard travel with it and come home after the last hop
 Only the exchange of K/V shards (and, in the backward, their gradient
 accumulators) crosses GPUs; the arithmetic of every step runs in the
 library's kernels. The contiguous sharding gives causal ranks unequal work
-(rank r computes r + 1 blocks).
+(rank r computes r + 1 blocks); the zig-zag layout at the end of this module
+(rank r holds sequence chunks r and 2R-1-r) gives every rank the same work.
+The exchange only ever sends the caller's K/V tensors: shards are received
+into two spare buffers used in turn.
 """
 
 from __future__ import annotations
@@ -87,19 +90,22 @@ def ring_exchange(k, v, group=None):
     r = dist.get_rank(group)
     nxt = dist.get_global_rank(group, (r + 1) % R) if group is not None else (r + 1) % R
     prv = dist.get_global_rank(group, (r - 1) % R) if group is not None else (r - 1) % R
+    # receive buffers: two, used in turn, so that the caller's k and v are
+    # only ever sent, never overwritten
     cur = (k, v)
-    spare = (torch.empty_like(k), torch.empty_like(v)) if R > 1 else None
+    spares = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, R - 1))]
     for t in range(R):
         reqs = []
         if t + 1 < R:
+            into = spares[t % len(spares)]
             ops = [dist.P2POp(dist.isend, cur[0], nxt, group), dist.P2POp(dist.isend, cur[1], nxt, group),
-                   dist.P2POp(dist.irecv, spare[0], prv, group), dist.P2POp(dist.irecv, spare[1], prv, group)]
+                   dist.P2POp(dist.irecv, into[0], prv, group), dist.P2POp(dist.irecv, into[1], prv, group)]
             reqs = dist.batch_isend_irecv(ops)
         yield (r - t) % R, cur[0], cur[1]
         for req in reqs:
             req.wait()
         if t + 1 < R:
-            cur, spare = spare, cur
+            cur = into
 
 
 class _GpuRank:
@@ -224,10 +230,12 @@ def ring_backward(k, v, rank: int, world: int, causal: bool, block_grad, new_acc
     sched = ring_schedule(rank, world, causal)
     cur = [k, v]
     acc = [new_acc(k), new_acc(v)]
+    # K/V receive buffers used in turn (the caller's k, v are never overwritten)
+    spares = [[x.new_empty(x.shape) for x in cur] for _ in range(min(2, world - 1))]
     if world > 1:
-        spare = [x.new_empty(x.shape) for x in cur]
         acc_spare = [new_acc(k), new_acc(v)]
     for t, src, mode in sched:
+        spare = spares[t % len(spares)] if t + 1 < world else None
         kv_move = exchange(cur, spare) if t + 1 < world else None  # overlaps the block
         if mode != "skip":
             dk_t, dv_t = block_grad(cur[0], cur[1], mode == "causal")
@@ -238,7 +246,7 @@ def ring_backward(k, v, rank: int, world: int, causal: bool, block_grad, new_acc
             acc, acc_spare = acc_spare, acc
         if kv_move is not None:
             kv_move.wait()
-            cur, spare = spare, cur
+            cur = spare
     return acc[0], acc[1]
 
 
@@ -340,3 +348,269 @@ def ring_attention_bwd_local(q_shards, k_shards, v_shards, o_shards, lse_shards,
             add(acc_k[src], dk_t, t == 0)
             add(acc_v[src], dv_t, t == 0)
     return [(gs[r].dq(), to_bf16(acc_k[r]), to_bf16(acc_v[r])) for r in range(R)]
+
+
+# ---------------------------------------------------------------- zig-zag layout
+#
+# With the causal mask the contiguous shards give rank r r + 1 blocks of work
+# (rank R-1 does R times what rank 0 does). The zig-zag layout cuts the
+# sequence into 2R chunks of c = N / (2R) tokens and gives rank r chunks r and
+# 2R-1-r: every rank then holds one early and one late chunk, and for the
+# causal mask every hop after the first is exactly two full c x c blocks on
+# every rank (hop 0: two causal diagonal blocks and one full block), 2R
+# full-block equivalents per rank. Shards are chunk-major, [2, B, c, H, d]
+# (chunk 0 = the early one), so that each chunk is a contiguous [B, c, H, d]
+# input of the single-GPU kernels, which take equal query and key lengths:
+# every block of the ring is one c x c call.
+
+
+def zigzag_chunks(rank: int, world: int):
+    """Global indices (of the 2R chunks of the sequence) of the two chunks rank holds."""
+    return rank, 2 * world - 1 - rank
+
+
+def chunk_mode(q_chunk: int, k_chunk: int, causal: bool) -> str:
+    """How query chunk q_chunk attends key chunk k_chunk (global chunk indices)."""
+    if not causal or k_chunk < q_chunk:
+        return "full"
+    if k_chunk == q_chunk:
+        return "causal"
+    return "skip"
+
+
+def zigzag_schedule(rank: int, world: int, causal: bool):
+    """[(hop, source rank of the K/V shard, [(i, j, mode), ...])] for one rank:
+    local query chunk i (0 early, 1 late) against chunk j of the held shard,
+    skipped pairs left out, in the order they are computed."""
+    mine = zigzag_chunks(rank, world)
+    out = []
+    for t in range(world):
+        src = (rank - t) % world
+        theirs = zigzag_chunks(src, world)
+        pairs = [(i, j, chunk_mode(mine[i], theirs[j], causal)) for i in range(2) for j in range(2)]
+        out.append((t, src, [p for p in pairs if p[2] != "skip"]))
+    return out
+
+
+def zigzag_shard(x, rank: int, world: int):
+    """[B, N, H, d] -> this rank's chunk-major zig-zag shard [2, B, N/(2R), H, d]."""
+    import torch
+    B, N, H, d = x.shape
+    if N % (2 * world):
+        raise ValueError(f"N = {N} is not a multiple of 2 x {world} ranks")
+    c = N // (2 * world)
+    a, b = zigzag_chunks(rank, world)
+    return torch.stack([x[:, a * c:(a + 1) * c], x[:, b * c:(b + 1) * c]]).contiguous()
+
+
+def zigzag_unshard(shards):
+    """Per-rank chunk-major shards [2, B, c, H, d] -> the whole sequence [B, 2Rc, H, d]."""
+    import torch
+    R = len(shards)
+    chunks = [None] * (2 * R)
+    for r, s in enumerate(shards):
+        a, b = zigzag_chunks(r, R)
+        chunks[a], chunks[b] = s[0], s[1]
+    return torch.cat(chunks, dim=1)
+
+
+def zigzag_unshard_lse(shards):
+    """Per-rank [2, B, H, c] LSE shards -> [B, H, 2Rc]."""
+    import torch
+    R = len(shards)
+    chunks = [None] * (2 * R)
+    for r, s in enumerate(shards):
+        a, b = zigzag_chunks(r, R)
+        chunks[a], chunks[b] = s[0], s[1]
+    return torch.cat(chunks, dim=-1)
+
+
+def zigzag_forward(q_chunks, kv_blocks, rank: int, world: int, causal: bool, block_attention, merge):
+    """Transport-agnostic core of the zig-zag ring.
+
+    q_chunks = (early, late) query chunks of this rank; kv_blocks yields
+    (src, k, v) in hop order with k, v indexable by chunk (0, 1);
+    block_attention(i, q, k, v, causal) -> (O, LSE) of one c x c block of
+    query chunk i;
+    merge(i, o, lse, first, last) folds a block into query chunk i's result
+    and returns that result after the chunk's last block. Returns
+    [result of chunk 0, result of chunk 1]."""
+    sched = zigzag_schedule(rank, world, causal)
+    last = {}
+    for t, _, pairs in sched:
+        for p, (i, _, _) in enumerate(pairs):
+            last[i] = (t, p)
+    seen, out = set(), [None, None]
+    for t, (src, k, v) in enumerate(kv_blocks):
+        if src != sched[t][1]:
+            raise RuntimeError(f"ring order broken: hop {t} holds shard {src}, expected {sched[t][1]}")
+        for p, (i, j, mode) in enumerate(sched[t][2]):
+            o_t, lse_t = block_attention(i, q_chunks[i], k[j], v[j], mode == "causal")
+            res = merge(i, o_t, lse_t, i not in seen, last[i] == (t, p))
+            seen.add(i)
+            if res is not None:
+                out[i] = res
+    return out
+
+
+def zigzag_backward(k, v, rank: int, world: int, causal: bool, block_grad, new_acc, add, exchange):
+    """Transport-agnostic zig-zag ring backward for one rank.
+
+    k, v: this rank's chunk-major shards; block_grad(i, kk, vv, causal) ->
+    (dk_t, dv_t) of query chunk i against one key chunk (it folds its own dq
+    contribution in); new_acc(x) -> an accumulator shaped like x (chunk-major,
+    it travels with its shard); add(acc, part, first) sets or adds in place;
+    exchange(send, recv) -> handle. Returns (dk_acc, dv_acc) of this rank's
+    own shard."""
+    sched = zigzag_schedule(rank, world, causal)
+    cur = [k, v]
+    acc = [new_acc(k), new_acc(v)]
+    # K/V receive buffers used in turn (the caller's k, v are never overwritten)
+    spares = [[x.new_empty(x.shape) for x in cur] for _ in range(min(2, world - 1))]
+    if world > 1:
+        acc_spare = [new_acc(k), new_acc(v)]
+    for t, src, pairs in sched:
+        spare = spares[t % len(spares)] if t + 1 < world else None
+        kv_move = exchange(cur, spare) if t + 1 < world else None  # overlaps the blocks
+        started = set()
+        for i, j, mode in pairs:
+            dk_t, dv_t = block_grad(i, cur[0][j], cur[1][j], mode == "causal")
+            first = t == 0 and j not in started  # hop 0 is the own shard: both chunks get a block
+            add(acc[0][j], dk_t, first)
+            add(acc[1][j], dv_t, first)
+            started.add(j)
+        if world > 1:  # the accumulators follow their shard (home after the last hop)
+            exchange(acc, acc_spare).wait()
+            acc, acc_spare = acc_spare, acc
+        if kv_move is not None:
+            kv_move.wait()
+            cur = spare
+    return acc[0], acc[1]
+
+
+class _GpuZigzag:
+    """The GPU side of one rank's zig-zag ring forward: each block of query
+    chunk i writes its bf16 (O, LSE) into the next of chunk i's slots, and
+    after the chunk's last block one merge kernel combines its slots."""
+
+    def __init__(self, q, rank, world, causal, scale):
+        import torch
+        _, B, c, H, d = q.shape
+        self.dims = (B, c, H, d)
+        self.scale = scale
+        counts = [0, 0]
+        for _, _, pairs in zigzag_schedule(rank, world, causal):
+            for i, _, _ in pairs:
+                counts[i] += 1
+        self.counts = counts
+        self.o_parts = [torch.empty((n, B, c, H, d), dtype=torch.bfloat16, device=q.device) for n in counts]
+        self.lse_parts = [torch.empty((n, B, H, c), dtype=torch.float32, device=q.device) for n in counts]
+        self.o = torch.empty((2, B, c, H, d), dtype=torch.bfloat16, device=q.device)
+        self.lse = torch.empty((2, B, H, c), dtype=torch.float32, device=q.device)
+        self.used = [0, 0]
+
+    def block(self, i, q, k, v, causal):
+        from . import attention_fwd
+        n = self.used[i]
+        self.used[i] += 1
+        return attention_fwd(q, k, v, causal=causal, scale=self.scale, out=self.o_parts[i][n],
+                             lse=self.lse_parts[i][n])
+
+    def merge(self, i, o_t, lse_t, first, last):
+        from . import fa_attn_merge
+        if not last:
+            return None
+        B, c, H, d = self.dims
+        if self.counts[i] == 1:
+            self.o[i].copy_(self.o_parts[i][0])
+            self.lse[i].copy_(self.lse_parts[i][0])
+        else:
+            fa_attn_merge(self.o_parts[i], self.lse_parts[i], self.counts[i], self.o[i], self.lse[i], B, c, H, d)
+        return True
+
+
+def _zigzag_fwd_rank(q, kv_blocks, rank, world, causal, scale):
+    g = _GpuZigzag(q, rank, world, causal, scale)
+    zigzag_forward((q[0], q[1]), kv_blocks, rank, world, causal, g.block, g.merge)
+    return g.o, g.lse
+
+
+def ring_attention_fwd_zigzag(q, k, v, causal=True, scale=None, group=None):
+    """Zig-zag sequence-parallel exact attention over the ranks of `group`.
+
+    q [2, B, c, Hq, d], k, v [2, B, c, Hkv, d] bf16 on this rank's GPU: this
+    rank's chunks (zigzag_shard) of sequences of length 2Rc. Returns
+    (o [2, B, c, Hq, d] bf16, lse [2, B, Hq, c] fp32) for this rank's query
+    rows over all keys of the sequence."""
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    return _zigzag_fwd_rank(q, ring_exchange(k, v, group), r, R, causal, scale)
+
+
+def ring_attention_fwd_zigzag_local(q_shards, k_shards, v_shards, causal=True, scale=None):
+    """The zig-zag ring of R ranks run by one process on one GPU (shard r of
+    each list plays rank r, hop t reads shard (r - t) mod R from the lists).
+    Same blocks, kernels and merge order as ring_attention_fwd_zigzag.
+    Returns per-rank (o, lse)."""
+    R = len(q_shards)
+    scale = 1.0 / math.sqrt(q_shards[0].shape[-1]) if scale is None else scale
+    outs = []
+    for r in range(R):
+        blocks = (((r - t) % R, k_shards[(r - t) % R], v_shards[(r - t) % R]) for t in range(R))
+        outs.append(_zigzag_fwd_rank(q_shards[r], blocks, r, R, causal, scale))
+    return outs
+
+
+def _zigzag_bwd_rank(q, k, v, o, lse, do, rank, world, causal, scale, exchange):
+    import torch
+    new_acc, add, to_bf16 = _gpu_acc_ops()
+    gs = [_GpuRankBwd(q[i], o[i], lse[i], do[i], k.shape[3], scale) for i in range(2)]
+
+    def block_grad(i, kk, vv, c):
+        return gs[i].block(kk, vv, c)
+
+    dk, dv = zigzag_backward(k, v, rank, world, causal, block_grad, new_acc, add, exchange)
+    return torch.stack([gs[0].dq(), gs[1].dq()]), to_bf16(dk), to_bf16(dv)
+
+
+def ring_attention_bwd_zigzag(q, k, v, o, lse, do, causal=True, scale=None, group=None):
+    """Gradients of zig-zag ring attention over the ranks of `group`: this
+    rank's chunk-major shards q, do, o [2,B,c,Hq,d], lse [2,B,Hq,c] (from
+    ring_attention_fwd_zigzag) and k, v [2,B,c,Hkv,d] -> (dq, dk, dv) bf16,
+    chunk-major, for this rank's shards."""
+    import torch.distributed as dist
+
+    R = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    return _zigzag_bwd_rank(q, k, v, o, lse, do, r, R, causal, scale, _p2p_exchange(group))
+
+
+def ring_attention_bwd_zigzag_local(q_shards, k_shards, v_shards, o_shards, lse_shards, do_shards, causal=True,
+                                    scale=None):
+    """The zig-zag ring backward of R ranks run by one process on one GPU,
+    hop by hop (at hop t every rank r works on shard (r - t) mod R, whose
+    accumulators receive their partials in the same order as on the ring).
+    Returns per-rank (dq, dk, dv), chunk-major."""
+    import torch
+    R = len(q_shards)
+    scale = 1.0 / math.sqrt(q_shards[0].shape[-1]) if scale is None else scale
+    new_acc, add, to_bf16 = _gpu_acc_ops()
+    gs = [[_GpuRankBwd(q_shards[r][i], o_shards[r][i], lse_shards[r][i], do_shards[r][i], k_shards[r].shape[3],
+                       scale) for i in range(2)] for r in range(R)]
+    acc_k = [new_acc(x) for x in k_shards]
+    acc_v = [new_acc(x) for x in v_shards]
+    for t in range(R):
+        for r in range(R):
+            src = (r - t) % R
+            started = set()
+            for i, j, mode in zigzag_schedule(r, R, causal)[t][2]:
+                dk_t, dv_t = gs[r][i].block(k_shards[src][j], v_shards[src][j], mode == "causal")
+                first = t == 0 and j not in started
+                add(acc_k[src][j], dk_t, first)
+                add(acc_v[src][j], dv_t, first)
+                started.add(j)
+    return [(torch.stack([gs[r][0].dq(), gs[r][1].dq()]), to_bf16(acc_k[r]), to_bf16(acc_v[r])) for r in range(R)]

@@ -4,7 +4,7 @@
   the oracle's LSE merge of key partitions on the same values: LSE within
   1e-5, the bf16 O within the bf16 bounds; rows no partial saw: O = 0,
   LSE = -inf.
-* The ring: R ranks played by one process on one GPU
+* The ring (contiguous and zig-zag layouts): R ranks played by one process on one GPU
   (`ring_attention_fwd_local`: the same blocks, kernels and merge order as the
   NCCL ring) against exact attention over the whole sequence; bounds of the
   bf16 forward (O max-abs <= 2e-2, relative RMS <= 5e-3, |dLSE| <= 1e-3).
@@ -104,5 +104,36 @@ def test_ring_backward_matches_full_gradient(fa, R, causal, Hq, Hkv, d):
     assert fa.fa_get_status() == fa.FA_OK
     dq, dk, dv = (torch.cat([g[i].cpu() for g in grads], dim=1).double().numpy() for i in range(3))
     dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, 1 / math.sqrt(d))
+    for got, ref in ((dq, dq_ref), (dk, dk_ref), (dv, dv_ref)):
+        assert oracle.rel_rms(got, ref) <= 1e-2
+
+
+@pytest.mark.parametrize("R", [1, 2, 4])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("Hq,Hkv,d", [(4, 2, 128), (2, 2, 64)])
+def test_zigzag_ring_fwd_bwd_match_full_attention(fa, R, causal, Hq, Hkv, d):
+    """The zig-zag layout (rank r holds chunks r and 2R-1-r), R ranks on one
+    GPU, forward then backward, against the oracle over the whole sequence:
+    the bf16 forward bounds and relative RMS <= 1e-2 per gradient. Chunks of
+    N/(2R) rows: several tiles and a ragged tail at R = 4 (1280/8 = 160)."""
+    from io_aware_exact_27_b200.ring import (ring_attention_bwd_zigzag_local, ring_attention_fwd_zigzag_local,
+                                             zigzag_shard, zigzag_unshard, zigzag_unshard_lse)
+    B, N = 2, 1280
+    q, k, v, do = synth.qkv_bf16(R * 13 + d, B, N, Hq, Hkv, d, with_dout=True)
+    dev = torch.device("cuda")
+    qs, ks, vs, dos = ([zigzag_shard(t, r, R).to(dev) for r in range(R)] for t in (q, k, v, do))
+    fw = ring_attention_fwd_zigzag_local(qs, ks, vs, causal=causal)
+    grads = ring_attention_bwd_zigzag_local(qs, ks, vs, [x[0] for x in fw], [x[1] for x in fw], dos, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    o = zigzag_unshard([x[0].cpu() for x in fw]).double().numpy()
+    lse = zigzag_unshard_lse([x[1].cpu() for x in fw]).double().numpy()
+    scale = 1 / math.sqrt(d)
+    O, L = oracle.attn_fwd(q, k, v, causal, scale)
+    assert oracle.max_abs(o, O) <= 2e-2
+    assert oracle.rel_rms(o, O) <= 5e-3
+    assert float(np.max(np.abs(lse - L))) <= 1e-3
+    dq, dk, dv = (zigzag_unshard([g[i].cpu() for g in grads]).double().numpy() for i in range(3))
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, scale)
     for got, ref in ((dq, dq_ref), (dk, dk_ref), (dv, dv_ref)):
         assert oracle.rel_rms(got, ref) <= 1e-2

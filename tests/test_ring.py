@@ -67,12 +67,14 @@ def _rank_main(rank, world, port, causal, B, N, Hq, Hkv, d, errs):
             o, l = oracle.merge_partials(parts_o, parts_l)
             return o, np.transpose(l, (0, 2, 1))
 
+        k_keep, v_keep = k_r.clone(), v_r.clone()
         O, L = ring_forward(q_r, ring_exchange(k_r, v_r), rank, world, causal, block, merge)
         O_ref, L_ref = oracle.attn_fwd(q, k, v, causal, scale)
         e_o = float(np.max(np.abs(O - O_ref[:, sl])))
         e_l = float(np.max(np.abs(L - L_ref[:, :, sl])))
-        if e_o > 1e-12 or e_l > 1e-12:
-            errs.put(f"rank {rank}: |dO| {e_o:.3g} |dLSE| {e_l:.3g}")
+        intact = torch.equal(k_r, k_keep) and torch.equal(v_r, v_keep)  # sent, never received into
+        if e_o > 1e-12 or e_l > 1e-12 or not intact:
+            errs.put(f"rank {rank}: |dO| {e_o:.3g} |dLSE| {e_l:.3g}, inputs intact: {intact}")
         else:
             errs.put(None)
     except Exception as e:  # reported to the parent
@@ -125,8 +127,11 @@ def _rank_bwd_main(rank, world, port, causal, B, N, Hq, Hkv, d, errs):
 
         k_r = torch.from_numpy(np.ascontiguousarray(k[:, sl]))
         v_r = torch.from_numpy(np.ascontiguousarray(v[:, sl]))
+        k_keep, v_keep = k_r.clone(), v_r.clone()
         dk, dv = ring_backward(k_r, v_r, rank, world, causal, block_grad, lambda x: torch.zeros_like(x), add,
                                _p2p_exchange())
+        if not (torch.equal(k_r, k_keep) and torch.equal(v_r, v_keep)):
+            raise RuntimeError("the ring overwrote the caller's K/V shard")
         dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, scale)
         e = max(float(np.abs(dq - dq_ref[:, sl]).max()), float(np.abs(dk.numpy() - dk_ref[:, sl]).max()),
                 float(np.abs(dv.numpy() - dv_ref[:, sl]).max()))
@@ -144,6 +149,136 @@ def test_ring_backward_on_cpu_ranks(world, causal):
     port = _free_port()
     B, N, Hq, Hkv, d = 2, 16 * world, 4, 2, 8
     procs = [ctx.Process(target=_rank_bwd_main, args=(r, world, port, causal, B, N, Hq, Hkv, d, errs))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [errs.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(r is None for r in results), results
+
+
+# ---------------------------------------------------------------- zig-zag layout
+
+from io_aware_exact_27_b200.ring import (chunk_mode, zigzag_backward, zigzag_chunks, zigzag_forward,  # noqa: E402
+                                         zigzag_schedule, zigzag_shard, zigzag_unshard)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 6])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_schedule_is_balanced_and_covers_each_pair_once(world, causal):
+    seen = {}
+    for r in range(world):
+        sched = zigzag_schedule(r, world, causal)
+        assert [t for t, _, _ in sched] == list(range(world))
+        assert sorted(src for _, src, _ in sched) == list(range(world))
+        mine = zigzag_chunks(r, world)
+        work = 0.0
+        for _, src, pairs in sched:
+            theirs = zigzag_chunks(src, world)
+            for i, j, mode in pairs:
+                key = (mine[i], theirs[j])
+                assert key not in seen
+                seen[key] = mode
+                assert mode == chunk_mode(mine[i], theirs[j], causal) != "skip"
+                work += 1.0 if mode == "full" else 0.5
+        # every rank: 2R full c x c blocks with the causal mask, 4R without
+        assert work == (2 * world if causal else 4 * world)
+    n = 2 * world
+    want = {(a, b) for a in range(n) for b in range(n) if not causal or b <= a}
+    assert set(seen) == want
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_zigzag_shard_round_trip(world):
+    x = torch.arange(2 * 12 * world * 3 * 2, dtype=torch.float32).reshape(2, 12 * world, 3, 2)
+    shards = [zigzag_shard(x, r, world) for r in range(world)]
+    assert all(s.shape == (2, 2, 6, 3, 2) for s in shards)
+    assert torch.equal(zigzag_unshard(shards), x)
+    with pytest.raises(ValueError):
+        zigzag_shard(x[:, :-1], 0, world)
+
+
+def _zigzag_chunks_np(x, rank, world, axis):
+    n = x.shape[axis] // (2 * world)
+    a, b = zigzag_chunks(rank, world)
+    take = lambda i: np.take(x, np.arange(i * n, (i + 1) * n), axis=axis)  # noqa: E731
+    return take(a), take(b)
+
+
+def _zz_rank_main(rank, world, port, causal, B, N, Hq, Hkv, d, errs):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(5)
+        q, k, v, do = (rng.standard_normal((B, N, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+        scale = 1.0 / math.sqrt(d)
+        O, L = oracle.attn_fwd(q, k, v, causal, scale)
+        qc = _zigzag_chunks_np(q, rank, world, 1)
+        kz = torch.from_numpy(np.stack(_zigzag_chunks_np(k, rank, world, 1)))
+        vz = torch.from_numpy(np.stack(_zigzag_chunks_np(v, rank, world, 1)))
+        parts = [([], []), ([], [])]
+
+        def block(i, qq, kk, vv, c):
+            return oracle.attn_fwd(qq, kk.numpy(), vv.numpy(), c, scale)
+
+        def merge(i, o_t, lse_t, first, last):
+            parts[i][0].append(o_t)
+            parts[i][1].append(np.transpose(lse_t, (0, 2, 1)))
+            if not last:
+                return None
+            o, l = oracle.merge_partials(*parts[i])
+            return o, np.transpose(l, (0, 2, 1))
+
+        res = zigzag_forward(qc, ring_exchange(kz, vz), rank, world, causal, block, merge)
+        e = 0.0
+        for i, (o_ref, l_ref) in enumerate(zip(_zigzag_chunks_np(O, rank, world, 1),
+                                              _zigzag_chunks_np(L, rank, world, 2))):
+            e = max(e, float(np.abs(res[i][0] - o_ref).max()), float(np.abs(res[i][1] - l_ref).max()))
+        e_fwd = e
+        # backward: the same ring with the oracle's block gradients
+        from io_aware_exact_27_b200.ring import _p2p_exchange
+        doc = _zigzag_chunks_np(do, rank, world, 1)
+        oc, lc = _zigzag_chunks_np(O, rank, world, 1), _zigzag_chunks_np(L, rank, world, 2)
+        dq = [np.zeros_like(x) for x in qc]
+
+        def block_grad(i, kk, vv, c):
+            a, bb, cc = oracle.attn_bwd_block(qc[i], kk.numpy(), vv.numpy(), doc[i], oc[i], lc[i], c, scale)
+            dq[i] += a
+            return torch.from_numpy(bb), torch.from_numpy(cc)
+
+        def add(acc, part, first):
+            if first:
+                acc.copy_(part)
+            else:
+                acc.add_(part)
+
+        dk, dv = zigzag_backward(kz, vz, rank, world, causal, block_grad, lambda x: torch.zeros_like(x), add,
+                                 _p2p_exchange())
+        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, scale)
+        for i in range(2):
+            e = max(e, float(np.abs(dq[i] - _zigzag_chunks_np(dq_ref, rank, world, 1)[i]).max()),
+                    float(np.abs(dk[i].numpy() - _zigzag_chunks_np(dk_ref, rank, world, 1)[i]).max()),
+                    float(np.abs(dv[i].numpy() - _zigzag_chunks_np(dv_ref, rank, world, 1)[i]).max()))
+        # the ring sends the caller's K/V shards but never receives into them
+        intact = np.array_equal(kz.numpy(), np.stack(_zigzag_chunks_np(k, rank, world, 1))) and \
+            np.array_equal(vz.numpy(), np.stack(_zigzag_chunks_np(v, rank, world, 1)))
+        errs.put(None if e <= 1e-12 and intact else
+                 f"rank {rank}: max error {e:.3g} (forward {e_fwd:.3g}), inputs intact: {intact}")
+    except Exception as ex:  # reported to the parent
+        errs.put(f"rank {rank}: {type(ex).__name__}: {ex}")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (2, False), (3, True)])
+def test_zigzag_ring_fwd_bwd_on_cpu_ranks(world, causal):
+    ctx = mp.get_context("spawn")
+    errs = ctx.Queue()
+    port = _free_port()
+    B, N, Hq, Hkv, d = 2, 12 * world, 4, 2, 8
+    procs = [ctx.Process(target=_zz_rank_main, args=(r, world, port, causal, B, N, Hq, Hkv, d, errs))
              for r in range(world)]
     for p in procs:
         p.start()
