@@ -1,5 +1,7 @@
 """The C-ABI library loads on a machine without a GPU and exports every entry
-point that include/fa_b200.h declares (no compute calls here)."""
+point that include/fa_b200.h declares; its pure host logic (workspace sizes,
+status strings, argument checks that return before any device work) answers
+there too. No compute calls here."""
 
 import ctypes
 import os
@@ -62,3 +64,31 @@ def test_binding_imports_and_names_match():
     import io_aware_exact_27_b200 as fa
     for name in declared_functions():
         assert hasattr(fa, name), f"binding lacks {name}"
+
+
+def test_kvcache_workspace_size_host_logic(lib):
+    """Split-KV decode scratch: per split, one fp32 partial O row (d floats)
+    and its LSE for every (batch, query, head); nothing for a single split."""
+    f = lib.fa_fwd_kvcache_workspace_size
+    f.restype = ctypes.c_size_t
+    assert f(16, 1, 32, 128, 1) == 0 and f(16, 1, 32, 128, 0) == 0
+    for B, Nq, Hq, d, s in ((16, 1, 32, 128, 4), (2, 3, 8, 64, 7)):
+        assert f(B, Nq, Hq, d, s) == s * B * Nq * Hq * (d + 1) * 4
+    assert f(0, 1, 32, 128, 4) == 0 and f(16, 1, 32, 128, 8) == 2 * f(16, 1, 32, 128, 4)
+
+
+def test_argument_checks_before_any_device_work(lib):
+    """Calls rejected (or empty) by their host-side checks return before
+    touching a device, so they answer on a machine without one."""
+    P = ctypes.c_void_p
+    lib.fa_fwd_blocksparse.argtypes = [P] * 6 + [ctypes.c_int] * 6 + [ctypes.c_float, P]
+    fake = P(16)
+    # negative sizes: invalid; an empty batch: nothing to do
+    assert lib.fa_fwd_blocksparse(fake, fake, fake, fake, fake, fake, -1, 1, 1, 128, 64, 0, 0.125, None) == 1
+    assert lib.fa_fwd_blocksparse(fake, fake, fake, fake, fake, fake, 0, 1, 1, 128, 64, 0, 0.125, None) == 0
+    # no mask: invalid; more than 1024 key blocks: unsupported
+    assert lib.fa_fwd_blocksparse(fake, fake, fake, None, fake, fake, 1, 1, 1, 128, 64, 0, 0.125, None) == 1
+    assert lib.fa_fwd_blocksparse(fake, fake, fake, fake, fake, fake, 1, 1, 1, 131073, 64, 0, 0.125, None) == 2
+    lib.fa_fwd.argtypes = [P] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float, P]
+    assert lib.fa_fwd(fake, fake, fake, fake, fake, -2, 1, 1, 128, 64, 0, 0.125, None) == 1
+    assert lib.fa_fwd(fake, fake, fake, fake, fake, 3, 1, 1, 0, 64, 0, 0.125, None) == 0
