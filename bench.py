@@ -179,6 +179,22 @@ class ClockSampler:
         return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
 
 
+def oracle_threads():
+    """Threads of the BLAS pool numpy runs the oracle's products on (the
+    cores the oracle actually uses; its elementwise steps run on one), and
+    that BLAS's name and version."""
+    try:
+        import numpy  # noqa: F401  (loads the BLAS the pool info reports)
+        import threadpoolctl
+        pools = [p for p in threadpoolctl.threadpool_info() if p.get("user_api") == "blas"]
+        if pools:
+            p = max(pools, key=lambda x: x.get("num_threads") or 0)
+            return int(p["num_threads"]), f"{p.get('internal_api')} {p.get('version')}"
+    except Exception:
+        pass
+    return os.cpu_count(), "unknown"
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -213,7 +229,7 @@ def oracle_sample(budget_s, with_bwd, w=None):
         if time.perf_counter() - t0 >= budget_s:
             break
     el = time.perf_counter() - t0
-    cores = os.cpu_count()
+    cores = oracle_threads()[0]
     return per_head * done / el / 1e12, done, el, cores
 
 
@@ -238,7 +254,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": dict(WORKLOAD, parallelism=f"replicas{args.gpus}", l2="n/a (CPU)"),
-            "cpu_baseline": {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1], "sample": sample},
             "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -413,7 +429,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, heads, el, cores = oracle_sample(args.cpu_budget_s, with_bwd)
-        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{heads} of {B * Hq} (batch, head) problems of the workload, fp64 numpy, "
                          f"{'fwd+bwd' if with_bwd else 'fwd'}, {el:.1f} s"}
 
@@ -470,7 +486,7 @@ def decode_oracle_sample(args, budget_s):
         done += 1
         if time.perf_counter() - t_start >= budget_s:
             break
-    return byts / B * done / el / 1e9, done, el, os.cpu_count()
+    return byts / B * done / el / 1e9, done, el, oracle_threads()[0]
 
 
 def run_decode_reference(args):
@@ -491,7 +507,7 @@ def run_decode_reference(args):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": dict(cfg, parallelism=f"replicas{args.gpus}", l2="n/a (CPU)"),
-            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": vals[-1][3], "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1], "sample": sample},
             "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -598,7 +614,7 @@ def run_decode(args):
     cpu = None
     if rank == 0 and world == 1:
         gbs, seqs, el, cores = decode_oracle_sample(args, args.cpu_budget_s)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{seqs} of {B} sequences of the workload, fp64 numpy, {el:.1f} s"}
     clocks = clk.summary()
     if pg:
@@ -800,7 +816,7 @@ def run_ring(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, rows, el, cores = ring_oracle_sample(args, args.cpu_budget_s)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{rows} query rows of head 0, fp64 numpy, {el:.1f} s"}
     if pg:
         pg.barrier()
@@ -837,7 +853,7 @@ def ring_oracle_sample(args, budget_s):
         el += time.perf_counter() - t0
         flops += float(sum(4.0 * (r + 1) * d for r in rows))
         done += 64
-    return flops / el / 1e12, done, el, os.cpu_count()
+    return flops / el / 1e12, done, el, oracle_threads()[0]
 
 
 def run_ring_reference(args):
@@ -854,7 +870,7 @@ def run_ring_reference(args):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": f"bf16 causal ring attention forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}",
                        "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1],
                              "sample": f"{vals[-1][1]} query rows of head 0 per step, fp64 numpy"},
             "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -1037,7 +1053,7 @@ def run_fp8(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, nr, el, cores = fp8_oracle_sample(args.cpu_budget_s)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{nr} (head, query row) pairs of the workload, fp64 numpy, {el:.1f} s"}
     clocks = clk.summary()
     if pg:
@@ -1083,7 +1099,7 @@ def fp8_oracle_sample(budget_s):
         el += time.perf_counter() - t0
         flops += float(sum(4.0 * (r + 1) * d for r in rows))
         done += 64
-    return flops / el / 1e12, done, el, os.cpu_count()
+    return flops / el / 1e12, done, el, oracle_threads()[0]
 
 
 def run_fp8_reference(args):
@@ -1100,7 +1116,7 @@ def run_fp8_reference(args):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": f"fp8-e4m3 causal forward, B={B} Hq=Hkv={H} N={N} d={d}, rotated Q/K",
                        "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1],
                              "sample": f"{vals[-1][1]} query rows of one head per step, fp64 numpy"},
             "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -1263,7 +1279,7 @@ def run_blocksparse(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, nr, el, cores = bs_oracle_sample(args.cpu_budget_s)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{nr} query rows of head 0, fp64 numpy, {el:.1f} s"}
     clocks = clk.summary()
     if pg:
@@ -1307,7 +1323,7 @@ def bs_oracle_sample(budget_s):
             flops += 4.0 * d * keys.size
         el += time.perf_counter() - t0
         done += 32
-    return flops / el / 1e12, done, el, os.cpu_count()
+    return flops / el / 1e12, done, el, oracle_threads()[0]
 
 
 def run_bs_reference(args):
@@ -1324,7 +1340,7 @@ def run_bs_reference(args):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": f"bf16 causal block-sparse forward, B={B} Hq={Hq} Hkv={Hkv} N={N} d={d}",
                        "parallelism": f"replicas{args.gpus}", "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle",
+            "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1],
                              "sample": f"{vals[-1][1]} query rows of head 0 per step, fp64 numpy"},
             "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -1364,7 +1380,7 @@ def run_sweep(args):
                           "data": "synthetic", "impl": "reference",
                           "config": {"workload": f"causal attention fwd+bwd sweep, N in {list(SWEEP_NS)}, "
                                                  f"B*N = {SWEEP_TOKENS}, Hq=Hkv={SWEEP_H}, d={SWEEP_D}"},
-                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle",
+                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1],
                                            "sample": sample},
                           "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
               flush=True)
@@ -1447,7 +1463,7 @@ def run_sweep(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, heads, el, cores = oracle_sample(args.cpu_budget_s, True, sweep_workload(SWEEP_NS[0]))
-        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{heads} (batch, head) problems of the N=2048 point, fp64 numpy, fwd+bwd, {el:.1f} s"}
     clocks = clk.summary()
     if pg:
@@ -1501,7 +1517,7 @@ def varlen_oracle_sample(budget_s, lengths, cu):
         if time.perf_counter() - t0 >= budget_s:
             break
     el = time.perf_counter() - t0
-    return flops / el / 1e12, done, el, os.cpu_count()
+    return flops / el / 1e12, done, el, oracle_threads()[0]
 
 
 def run_varlen(args):
@@ -1526,7 +1542,7 @@ def run_varlen(args):
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                           "data": "synthetic", "impl": "reference", "config": {"workload": wl},
-                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle",
+                          "cpu_baseline": {"value": tf, "unit": UNIT, "cores": vals[-1][3], "kind": "oracle", "blas": oracle_threads()[1],
                                            "sample": f"{vals[0][1]} (sequence, head) problems per step, fp64 "
                                                      f"numpy, fwd+bwd"},
                           "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
@@ -1625,7 +1641,7 @@ def run_varlen(args):
     cpu = None
     if rank == 0 and world == 1:
         tf, n, el, cores = varlen_oracle_sample(args.cpu_budget_s, lengths, cu_h)
-        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{n} of {nseq * H} (sequence, head) problems, fp64 numpy, fwd+bwd, {el:.1f} s"}
     clocks = clk.summary()
     if pg:

@@ -29,6 +29,7 @@ def test_reference_arm_prints_one_contract_line(workload):
     assert j["impl"] == "reference" and j["n_gpus"] == 1 and j["steps"] == 1
     assert j["value"] > 0 and j["cpu_baseline"]["value"] == j["value"]
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert isinstance(j["cpu_baseline"]["blas"], str)
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
     assert isinstance(j["config"]["workload"], str) and j["config"]["workload"]
 
