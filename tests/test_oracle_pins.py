@@ -573,3 +573,20 @@ def test_blocksparse_backward_pins():
         fd = (f(*args1) - f(*args2)) / (2 * eps)
         assert abs(fd - grad[idx]) < 1e-6
     assert np.all(dq[0, 6:12, 0] == 0)  # the empty query block has no gradient
+
+
+# ---------------------------------------------------------------- error metrics
+
+def test_error_metrics_by_hand():
+    """max-abs and relative RMS (reading 8) on worked values: the reference
+    is the second operand and the norm is over the whole tensor."""
+    x, y = np.array([1.0, -2.0, 3.0]), np.array([1.0, 1.0, 1.0])
+    assert oracle.max_abs(x, y) == 3.0  # |x + y| would give 4
+    assert oracle.max_abs(y, y) == 0.0 and oracle.max_abs(np.zeros(0), np.zeros(0)) == 0.0
+    y2 = np.array([[3.0, 4.0]])  # ||y|| = 5
+    assert abs(oracle.rel_rms(np.array([[3.0, 0.0]]), y2) - 0.8) < 1e-15  # ||x|| = 3 in the denominator: 4/3
+    assert oracle.rel_rms(y2, y2) == 0.0
+    assert abs(oracle.rel_rms(y2, 2 * y2) - 0.5) < 1e-15 and abs(oracle.rel_rms(2 * y2, y2) - 1.0) < 1e-15
+    # the whole tensor, not a mean of per-row ratios: rows [1,0] and [0,100], error 1 in row 0 only
+    ref = np.array([[1.0, 0.0], [0.0, 100.0]])
+    assert abs(oracle.rel_rms(ref + np.array([[1.0, 0.0], [0.0, 0.0]]), ref) - 1.0 / np.sqrt(10001.0)) < 1e-15
