@@ -161,6 +161,7 @@ def attention_fwd_blocksparse(q, k, v, block_mask, causal=False, scale=None, str
     """q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16, block_mask uint8 [Hq, ceil(N/128), ceil(N/128)] (CUDA)
     -> (o [B,N,Hq,d] bf16, lse [B,Hq,N] f32)."""
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v), u8=dict(block_mask=block_mask))
     B, N, Hq, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
@@ -179,6 +180,7 @@ def attention_bwd_blocksparse(q, k, v, block_mask, o, lse, dout, causal=False, s
                               stream=None):
     """Gradients (dq, dk, dv) of sum(o * dout) for attention_fwd_blocksparse with the same block_mask."""
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, o=o, dout=dout), f32=dict(lse=lse), u8=dict(block_mask=block_mask))
     B, N, Hq, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = fa_bwd_blocksparse_workspace_size(B, Hq, k.shape[2], N, d)
@@ -202,6 +204,7 @@ def fa_fp8_quantize(x, codes, scales, B, N, H, d, rotate, stream=None):
 def quantize_fp8(x, rotate=False, stream=None):
     """x [B,N,H,d] bf16 (CUDA) -> (codes [B,N,H,d] float8_e4m3fn, scales [B,H,ceil(N/128)] f32)."""
     import torch
+    _check_inputs(bf16=dict(x=x))
     B, N, H, d = x.shape
     codes = torch.empty((B, N, H, d), dtype=torch.float8_e4m3fn, device=x.device)
     scales = torch.empty((B, H, (N + 127) // 128), dtype=torch.float32, device=x.device)
@@ -218,6 +221,7 @@ def dequantize_fp8(codes, scales, unrotate=False, stream=None):
     """codes [B,N,H,d] float8_e4m3fn + scales [B,H,ceil(N/128)] f32 (CUDA) -> bf16 [B,N,H,d]
     values in the original space (rotation undone with unrotate=True)."""
     import torch
+    _check_inputs(bytes1=dict(codes=codes), f32=dict(scales=scales))
     B, N, H, d = codes.shape
     x = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=codes.device)
     fa_fp8_dequantize(codes, scales, x, B, N, H, d, unrotate, stream)
@@ -301,9 +305,35 @@ def _default_scale(d, scale):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
+def _check_inputs(bf16=None, f32=None, i32=None, u8=None, bytes1=None):
+    """The C entry points see only data pointers: every tensor handed to them
+    must be dense (contiguous), of the documented element type, and on the
+    GPU. Each argument maps names to tensors of one element type (bytes1: any
+    1-byte type, the e4m3 codes). Layout and types are checked for all of
+    them before residency. Raises ValueError."""
+    import torch
+    groups = ((bf16, torch.bfloat16, None), (f32, torch.float32, None), (i32, torch.int32, None),
+              (u8, torch.uint8, None), (bytes1, None, 1))
+    named = []
+    for tensors, dtype, itemsize in groups:
+        for name, t in (tensors or {}).items():
+            if not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous (the library reads it as a dense array)")
+            if dtype is not None and t.dtype != dtype:
+                raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+            if itemsize is not None and t.element_size() != itemsize:
+                raise ValueError(f"{name} must have {itemsize}-byte elements, got {t.element_size()}")
+            named.append((name, t))
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+
+
 def attention_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
     """q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 CUDA tensors -> (o [B,N,Hq,d] bf16, lse [B,Hq,N] f32)."""
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, out=q if out is None else out),
+                  f32=None if lse is None else dict(lse=lse))
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     o = torch.empty_like(q) if out is None else out
@@ -316,6 +346,8 @@ def attention_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, scale=No
                          stream=None):
     """q [T,Hq,d], k/v [T,Hkv,d] bf16, cu_seqlens int32 [nseq+1] (CUDA) -> (o [T,Hq,d], lse [Hq,T])."""
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, out=q if out is None else out),
+                  f32=None if lse is None else dict(lse=lse), i32=dict(cu_seqlens=cu_seqlens))
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     o = torch.empty_like(q) if out is None else out
@@ -328,6 +360,7 @@ def attention_fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, scale=No
 def attention_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None, stream=None):
     """e4m3 q8 [B,N,Hq,d], k8/v8 [B,N,Hkv,d] + f32 block scales -> (o bf16, lse f32)."""
     import torch
+    _check_inputs(bytes1=dict(q8=q8, k8=k8, v8=v8), f32=dict(q_scale=q_scale, k_scale=k_scale, v_scale=v_scale))
     B, N, Hq, d = q8.shape
     Hkv = k8.shape[2]
     o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device=q8.device)
@@ -340,6 +373,7 @@ def attention_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale
 def attention_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, stream=None):
     """Gradients (dq, dk, dv) of sum(o * dout); inputs as attention_fwd produced them."""
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, o=o, dout=dout), f32=dict(lse=lse))
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -354,6 +388,7 @@ def attention_bwd(q, k, v, o, lse, dout, causal=False, scale=None, workspace=Non
 def attention_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen, causal=False, scale=None, workspace=None,
                          stream=None):
     import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, o=o, dout=dout), f32=dict(lse=lse), i32=dict(cu_seqlens=cu_seqlens))
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     nseq = cu_seqlens.numel() - 1
@@ -372,6 +407,7 @@ def attention_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, causal=True, scale
     -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] f32). num_splits defaults to the
     library's choice for this device (fa_fwd_kvcache_num_splits)."""
     import torch
+    _check_inputs(bf16=dict(q=q, k_cache=k_cache, v_cache=v_cache), i32=dict(cache_seqlens=cache_seqlens))
     B, Nq, Hq, d = q.shape
     Ncache, Hkv = k_cache.shape[1], k_cache.shape[2]
     if num_splits is None:

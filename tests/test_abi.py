@@ -92,3 +92,27 @@ def test_argument_checks_before_any_device_work(lib):
     lib.fa_fwd.argtypes = [P] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float, P]
     assert lib.fa_fwd(fake, fake, fake, fake, fake, -2, 1, 1, 128, 64, 0, 0.125, None) == 1
     assert lib.fa_fwd(fake, fake, fake, fake, fake, 3, 1, 1, 0, 64, 0, 0.125, None) == 0
+
+
+def test_torch_wrappers_reject_what_the_library_cannot_read():
+    """The C entry points see only data pointers: the torch-level calls refuse
+    non-contiguous views, other element types and host tensors before any
+    library call (so this runs without a GPU)."""
+    import torch
+    import io_aware_exact_27_b200 as fa
+    x = torch.zeros((2, 256, 4, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="contiguous"):
+        fa.attention_fwd(x[:, ::2], x[:, ::2], x[:, ::2])
+    with pytest.raises(ValueError, match="bfloat16"):
+        fa.attention_fwd(x.float(), x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.attention_fwd(x, x, x)
+    lse = torch.zeros((2, 4, 256), dtype=torch.float32)
+    with pytest.raises(ValueError, match="float32"):
+        fa.attention_bwd(x, x, x, x, lse.double(), x)
+    with pytest.raises(ValueError, match="int32"):
+        fa.attention_fwd_varlen(x[0], x[0], x[0], torch.zeros(3, dtype=torch.int64), 128)
+    with pytest.raises(ValueError, match="uint8"):
+        fa.attention_fwd_blocksparse(x, x, x, torch.ones((4, 2, 2), dtype=torch.int32))
+    with pytest.raises(ValueError, match="1-byte"):
+        fa.attention_fwd_fp8(x, x, x, lse, lse, lse)
