@@ -286,3 +286,78 @@ def test_zigzag_ring_fwd_bwd_on_cpu_ranks(world, causal):
     for p in procs:
         p.join(timeout=60)
     assert all(r is None for r in results), results
+
+
+def _sub_rank_main(rank, world, port, errs):
+    """Ranks 1 and 2 of 3 run the ring on a sub-group (group-local ranks 0 and
+    1); rank 0 only takes part in creating the group."""
+    from io_aware_exact_27_b200.ring import _p2p_exchange, ring_backward
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sub = dist.new_group([1, 2])
+        if rank == 0:
+            errs.put(None)
+            return
+        r, R = dist.get_rank(sub), dist.get_world_size(sub)
+        B, N, H, d, causal = 1, 16, 2, 8, True
+        rng = np.random.default_rng(9)
+        q, k, v, do = (rng.standard_normal((B, N, H, d)) for _ in range(4))
+        scale = 1.0 / math.sqrt(d)
+        n = N // R
+        sl = slice(r * n, (r + 1) * n)
+        k_r, v_r = torch.from_numpy(np.ascontiguousarray(k[:, sl])), torch.from_numpy(np.ascontiguousarray(v[:, sl]))
+        parts_o, parts_l = [], []
+
+        def block(qq, kk, vv, c):
+            return oracle.attn_fwd(qq, kk.numpy(), vv.numpy(), c, scale)
+
+        def merge(o_t, lse_t, first, last):
+            parts_o.append(o_t)
+            parts_l.append(np.transpose(lse_t, (0, 2, 1)))
+            if not last:
+                return None
+            o, l = oracle.merge_partials(parts_o, parts_l)
+            return o, np.transpose(l, (0, 2, 1))
+
+        O, L = ring_forward(q[:, sl], ring_exchange(k_r, v_r, group=sub), r, R, causal, block, merge)
+        O_ref, L_ref = oracle.attn_fwd(q, k, v, causal, scale)
+        e = max(float(np.abs(O - O_ref[:, sl]).max()), float(np.abs(L - L_ref[:, :, sl]).max()))
+        dq = np.zeros_like(q[:, sl])
+
+        def block_grad(kk, vv, c):
+            a, bb, cc = oracle.attn_bwd_block(q[:, sl], kk.numpy(), vv.numpy(), do[:, sl], O_ref[:, sl],
+                                              L_ref[:, :, sl], c, scale)
+            dq[...] += a
+            return torch.from_numpy(bb), torch.from_numpy(cc)
+
+        def add(acc, part, first):
+            if first:
+                acc.copy_(part)
+            else:
+                acc.add_(part)
+
+        dk, dv = ring_backward(k_r, v_r, r, R, causal, block_grad, lambda x: torch.zeros_like(x), add,
+                               _p2p_exchange(sub))
+        g = oracle.attn_bwd(q, k, v, do, causal, scale)
+        e = max(e, float(np.abs(dq - g[0][:, sl]).max()), float(np.abs(dk.numpy() - g[1][:, sl]).max()),
+                float(np.abs(dv.numpy() - g[2][:, sl]).max()))
+        errs.put(None if e <= 1e-12 else f"rank {rank} (group rank {r}): max error {e:.3g}")
+    except Exception as ex:  # reported to the parent
+        errs.put(f"rank {rank}: {type(ex).__name__}: {ex}")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_on_a_sub_group():
+    ctx = mp.get_context("spawn")
+    errs = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sub_rank_main, args=(r, 3, port, errs)) for r in range(3)]
+    for p in procs:
+        p.start()
+    results = [errs.get(timeout=120) for _ in range(3)]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(r is None for r in results), results
