@@ -195,6 +195,19 @@ def oracle_threads():
     return os.cpu_count(), "unknown"
 
 
+def max_over_ranks(pg, dev, value):
+    """The largest of `value` over the ranks of the default process group
+    (every rank calls this at the same point, with its own value): the
+    time of a multi-GPU run is its slowest rank's. pg is torch.distributed,
+    or None for a single process (value returned as is)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -350,10 +363,7 @@ def run_ours(args):
                 e[2 + j].record(stream)
     torch.cuda.synchronize(dev)
     seg = [[e[j].elapsed_time(e[j + 1]) for e in ev2] for j in range(nev - 1)]
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     ms_per_step = tot_ms / args.steps
     f_fwd = fwd_flops(B, Hq, N, d, causal)
     f_step = f_fwd * (3.5 if with_bwd else 1.0)
@@ -419,10 +429,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": f_step * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
@@ -572,10 +579,7 @@ def run_decode(args):
     if st != fa.FA_OK:
         raise SystemExit(f"device status error: {fa.fa_status_string(st)}")
     tot_ms = ev[0].elapsed_time(ev[-1])
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     ms_per_step = tot_ms / args.steps
     value = byts * world * args.steps / (tot_ms * 1e-3) / 1e9
     pk = peaks()
@@ -603,10 +607,7 @@ def run_decode(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": byts * world * args.e2e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": q_pin.numel() * 2 + lens_pin.numel() * 4,
                "d2h_bytes_per_step": o_pin.numel() * 2 + lse_pin.numel() * 4,
@@ -728,10 +729,7 @@ def run_ring(args):
         torch.cuda.synchronize(dev)
     timing["on"] = False
     tot_ms = e_beg.elapsed_time(e_end)
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     f_job = fwd_flops(B, Hq, N, d, True)  # the whole sequence's causal attention
     value = f_job * args.steps / (tot_ms * 1e-3) / 1e12
     k_ms = sum(a.elapsed_time(b) for a, b, _ in rec)
@@ -772,10 +770,7 @@ def run_ring(args):
         b1.record(stream)
         torch.cuda.synchronize(dev)
         b_ms = b0.elapsed_time(b1)
-        if pg:
-            t = torch.tensor([b_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            b_ms = float(t.item())
+        b_ms = max_over_ranks(pg, dev, b_ms)
         bwd = {"ms_per_step": b_ms / args.steps,
                "tflops": 2.5 * f_job * args.steps / (b_ms * 1e-3) / 1e12,
                "note": "ring backward timed separately: flops 2.5x the forward (five GEMMs)"}
@@ -805,10 +800,7 @@ def run_ring(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(pg, dev, e_ms)
         h2d = sum(x.numel() * x.element_size() for r in mine for x in pin[r])
         d2h = sum(x.numel() * x.element_size() for r in mine for x in outs_h[r])
         e2e = {"value": f_job * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -1006,10 +998,7 @@ def run_fp8(args):
     b_ms = sum(b0.elapsed_time(b1) for b0, b1 in bev) / args.steps
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error in the backward")
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     flops = fwd_flops(B, H, N, d, True)
     value = flops * world * args.steps / (tot_ms * 1e-3) / 1e12
     pk = peaks()
@@ -1043,10 +1032,7 @@ def run_fp8(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": flops * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": sum(x.numel() * 2 for x in pin),
                "d2h_bytes_per_step": o_h.numel() * 2 + l_h.numel() * 4}
@@ -1243,10 +1229,7 @@ def run_blocksparse(args):
     bwd = {"ms": b_ms, "tflops": 2.5 * flops / (b_ms * 1e-3) / 1e12, "dense_causal_ms": bd_ms,
            "speedup_vs_dense_causal": bd_ms / b_ms,
            "note": "fa_bwd_blocksparse (pre + dK/dV + dQ) on the same mask, per GPU; flops 2.5x the forward's"}
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     ms = tot_ms / args.steps
     value = flops * world / (ms * 1e-3) / 1e12
     pk = peaks()
@@ -1455,10 +1438,7 @@ def run_sweep(args):
     tiny_bytes = (2 * B * N * Hq * d + 2 * B * N * Hkv * d) * 2 + B * Hq * N * 4  # Q, K, V read; O, LSE written
     tiny = {"B": B, "Hq": Hq, "N": N, "d": d, "causal": causal, "fwd_us": ms_f * 1e3, "step_us": ms_s * 1e3,
             "fwd_gbs": tiny_bytes / (ms_f * 1e-3) / 1e9}
-    if pg:
-        t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        tot_ms = float(t.item())
+    tot_ms = max_over_ranks(pg, dev, tot_ms)
     value = tot_flops * world / (tot_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1:
@@ -1601,10 +1581,7 @@ def run_varlen(args):
     if fa.fa_get_status(sptr) != fa.FA_OK:
         raise SystemExit("device status error")
     ms_s, ms_f = ms
-    if pg:
-        t = torch.tensor([ms_s, ms_f], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_s, ms_f = (float(x) for x in t.tolist())
+    ms_s, ms_f = max_over_ranks(pg, dev, ms_s), max_over_ranks(pg, dev, ms_f)
     value = 3.5 * f * world / (ms_s * 1e-3) / 1e12
     pk = peaks()
     fwd_tf = f / (ms_f * 1e-3) / 1e12
@@ -1631,10 +1608,7 @@ def run_varlen(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": 3.5 * f * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)}

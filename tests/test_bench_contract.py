@@ -44,3 +44,39 @@ def test_traffic_lookup_is_keyed_by_shape():
         if e["source_hash"] == bench.kernel_source_hash(kernel):
             assert bench.traffic_for(kernel, e["shape"]) == e["dram_bytes_per_launch"]
         assert bench.traffic_for(kernel, e["shape"] + " other") is None
+
+
+def _max_rank_main(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(dist, torch.device("cpu"), 1.5 + 10.0 * rank)
+        again = bench.max_over_ranks(dist, torch.device("cpu"), 7.25 - rank)
+        q.put((rank, got, again))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_time_is_the_slowest_ranks_on_cpu_ranks():
+    """The multi-GPU bench reports each timed quantity as its maximum over the
+    ranks: gloo ranks stand in for the GPUs here."""
+    import socket
+    import torch.multiprocessing as mp
+    import bench
+    assert bench.max_over_ranks(None, None, 3.5) == 3.5
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_max_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+    assert res == [(0, 11.5, 7.25), (1, 11.5, 7.25)]
