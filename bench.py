@@ -88,10 +88,9 @@ KERNEL_HEADER = {"fa_fwd_sm100_kernel": "fa_fwd_kernel.cuh", "fa_bwd_dkdv_kernel
                  "fa_bwd_dq_kernel": "fa_bwd_kernel.cuh", "fa_decode_kernel": "fa_decode_kernel.cuh"}
 
 
-def kernel_source_hash(kernel):
-    """Hash of a kernel's device code: its header and every header it includes
-    (followed transitively). The host launcher is not part of it: a change of
-    a kernel's launch configuration there must be re-captured by hand."""
+def kernel_sources(kernel):
+    """The device sources of a profiled kernel: its header and every header it
+    includes, followed transitively (sorted names under csrc/)."""
     import re
     csrc = os.path.join(ROOT, "io_aware_exact_27_b200", "csrc")
     todo, seen = [KERNEL_HEADER[kernel]], []
@@ -101,6 +100,15 @@ def kernel_source_hash(kernel):
             continue
         seen.append(f)
         todo += re.findall(r'^#include "([^"]+)"', open(os.path.join(csrc, f)).read(), flags=re.M)
+    return sorted(seen)
+
+
+def kernel_source_hash(kernel):
+    """Hash of a kernel's device code (kernel_sources). The host launcher is
+    not part of it: a change of a kernel's launch configuration there must be
+    re-captured by hand."""
+    csrc = os.path.join(ROOT, "io_aware_exact_27_b200", "csrc")
+    seen = kernel_sources(kernel)
     h = hashlib.sha256()
     for f in sorted(seen):
         h.update(f.encode())

@@ -80,3 +80,17 @@ def test_time_is_the_slowest_ranks_on_cpu_ranks():
     for p in procs:
         p.join(timeout=60)
     assert res == [(0, 11.5, 7.25), (1, 11.5, 7.25)]
+
+
+def test_kernel_sources_keep_the_kernels_apart():
+    """A kernel's DRAM counters are keyed by its own device sources only: the
+    dK/dV and dQ kernels do not include the forward's or the preparation's
+    header, and the forward does not include the backward's."""
+    import bench
+    bwd = bench.kernel_sources("fa_bwd_dkdv_kernel")
+    assert bwd == bench.kernel_sources("fa_bwd_dq_kernel")
+    assert {"fa_bwd_kernel.cuh", "fa_bwd_args.cuh", "fa_tile.cuh", "fa_common.cuh", "sm100_ptx.cuh"} <= set(bwd)
+    assert "fa_fwd_kernel.cuh" not in bwd and "fa_bwd_pre_kernel.cuh" not in bwd
+    fwd = bench.kernel_sources("fa_fwd_sm100_kernel")
+    assert "fa_fwd_kernel.cuh" in fwd and not any(f.startswith("fa_bwd") for f in fwd)
+    assert "fa_decode_kernel.cuh" in bench.kernel_sources("fa_decode_kernel")
