@@ -35,6 +35,7 @@ from .attention import (  # noqa: F401
     attn_fwd_varlen,
     attn_bwd,
     attn_bwd_varlen,
+    attn_bwd_rows,
     attn_bwd_block,
     attn_fwd_kvcache,
     attn_fwd_blocksparse,

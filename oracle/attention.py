@@ -158,6 +158,42 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float):
     return dq, dk, dv
 
 
+def attn_bwd_rows(q, k, v, dout, causal: bool, scale: float, rows):
+    """Backward on a sample of query rows per head (long-context checks).
+
+    The same gradient as ``attn_bwd`` (the catalogue record's ``summary``:
+    recomputation of P from Q, K, V), restricted to the query rows ``rows``
+    [Hq, R] of each head (the same rows for every batch entry): for those
+    rows P, dP = dO V^T, D = rowsum(dO * O) and dS = P * (dP - D), then
+
+        dQ[rows] = scale dS K      (exact: a query row's gradient needs only its own row)
+        dK      += scale dS^T Q[rows],   dV += P^T dO[rows]   (the rows' share)
+
+    Returns dq [B,Hq,R,d] and the rows' contributions dk, dv [B,N,Hkv,d]
+    (float64; summed over the query heads of a kv head). Over a partition of
+    the rows the contributions sum to the full dK, dV (pinned)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    rows = np.asarray(rows, dtype=np.int64)
+    R = rows.shape[1]
+    dq = np.empty((B, Hq, R, d))
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            r = rows[h]
+            O, _, P = attention_head(q[b, :, h], k[b, :, g], v[b, :, g], causal, scale, r)
+            dP = do[b, r, h] @ v[b, :, g].T
+            D = (do[b, r, h] * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - D)
+            dq[b, h] = scale * (dS @ k[b, :, g])
+            dk[b, :, g] += scale * (dS.T @ q[b, r, h])
+            dv[b, :, g] += P.T @ do[b, r, h]
+    return dq, dk, dv
+
+
 def attn_bwd_varlen(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
     """Packed (varlen) backward: q, dout [T,Hq,d]; k, v [T,Hkv,d]."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)

@@ -236,6 +236,51 @@ def test_sampled_rows_match_full():
         np.testing.assert_allclose(Lr[:, h], L[:, h, rows[h]], atol=1e-14)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_backward_against_autograd(causal):
+    """attn_bwd_rows: torch fp64 SDPA autograd with dO zeroed outside each
+    head's sampled rows gives the sampled rows' dQ and exactly their share of
+    dK, dV (a query row's dQ needs only its own dO row)."""
+    B, N, Hq, Hkv, d, scale = 2, 40, 4, 2, 8, 0.35
+    q, k, v = _rand((B, N, Hq, d), 60), _rand((B, N, Hkv, d), 61), _rand((B, N, Hkv, d), 62)
+    do = _rand((B, N, Hq, d), 63)
+    rows = synth.sample_rows(1, N, Hq, R=9)
+    dq, dk, dv = oracle.attn_bwd_rows(q, k, v, do, causal, scale, rows)
+    keep = np.zeros((N, Hq))
+    for h in range(Hq):
+        keep[rows[h], h] = 1.0
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64).transpose(1, 2).requires_grad_() for x in (q, k, v))
+    rep = Hq // Hkv
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(rep, dim=1), tv.repeat_interleave(rep, dim=1), is_causal=causal, scale=scale)
+    to.backward(torch.tensor(do * keep[None, :, :, None]).transpose(1, 2))
+    gq = tq.grad.transpose(1, 2).numpy()
+    for h in range(Hq):
+        np.testing.assert_allclose(dq[:, h], gq[:, rows[h], h], atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.transpose(1, 2).numpy(), atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.transpose(1, 2).numpy(), atol=1e-12)
+
+
+def test_sampled_rows_backward_partition_sums_to_full():
+    """Over a partition of every head's rows the contributions add up to the
+    full gradient, and the rows' dQ are the full dQ's rows."""
+    B, N, Hq, Hkv, d, scale = 1, 24, 2, 1, 8, 0.4
+    q, k, v = _rand((B, N, Hq, d), 64), _rand((B, N, Hkv, d), 65), _rand((B, N, Hkv, d), 66)
+    do = _rand((B, N, Hq, d), 67)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, True, scale)
+    perm = np.random.default_rng(68).permutation(N)
+    parts = [np.stack([perm[:10]] * Hq), np.stack([perm[10:]] * Hq)]
+    sk, sv = np.zeros_like(dk), np.zeros_like(dv)
+    for rows in parts:
+        rq, rk, rv = oracle.attn_bwd_rows(q, k, v, do, True, scale, rows)
+        for h in range(Hq):
+            np.testing.assert_allclose(rq[:, h], dq[:, rows[h], h], atol=1e-13)
+        sk += rk
+        sv += rv
+    np.testing.assert_allclose(sk, dk, atol=1e-12)
+    np.testing.assert_allclose(sv, dv, atol=1e-12)
+
+
 def test_merge_partials_reproduces_full():
     N, d = 29, 8
     q, k, v = _rand((N, d), 49), _rand((N, d), 50), _rand((N, d), 51)
