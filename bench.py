@@ -2,10 +2,12 @@
 """Throughput of the exact-attention hot path on B200 (attention TFLOP/s).
 
 One step = the whole hot path over one batch of synthetic input: the causal
-bf16 forward pass (O, LSE) and, when the library provides it, the backward
-pass (dQ, dK, dV) on the workload B=4, Hq=Hkv=16, N=2048, d=128 (Q, K, V, dO
-i.i.d. N(0,1) rounded to bf16, seed 0). Flops: forward 4*B*Hq*N^2*d halved for
-causal, backward 2.5x the forward (five GEMMs instead of two).
+bf16 forward pass (O, LSE) and the backward pass (dQ, dK, dV). The default
+workload is long-context GQA attention, B=1 Hq=32 Hkv=8 N=16384 d=128
+(`--workload attention`); `--workload attention-2k` runs B=4 Hq=Hkv=16 N=2048
+d=128. Q, K, V, dO are i.i.d. N(0,1) rounded to bf16, seed 0 (rank r: seed r).
+Flops: forward 4*B*Hq*N^2*d halved for causal, backward 2.5x the forward
+(five GEMMs instead of two).
 
 The step is timed through the public calls (fa_fwd, fa_bwd); a second pass
 times the kernels one by one for the roofline of the dominant one.
@@ -30,8 +32,18 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = {"workload": "bf16 causal attention fwd+bwd, B=4 Hq=Hkv=16 N=2048 d=128",
-            "B": 4, "Hq": 16, "Hkv": 16, "N": 2048, "d": 128, "causal": True}
+# the two padded-batch fwd+bwd workloads; the first is the default line
+ATTN_WORKLOADS = {
+    "attention": {"workload": "bf16 causal attention fwd+bwd, long-context GQA, B=1 Hq=32 Hkv=8 N=16384 d=128",
+                  "B": 1, "Hq": 32, "Hkv": 8, "N": 16384, "d": 128, "causal": True},
+    "attention-2k": {"workload": "bf16 causal attention fwd+bwd, B=4 Hq=Hkv=16 N=2048 d=128",
+                     "B": 4, "Hq": 16, "Hkv": 16, "N": 2048, "d": 128, "causal": True},
+}
+WORKLOAD = dict(ATTN_WORKLOADS["attention"])
+# above this sequence length the CPU oracle samples query rows of a head
+# instead of whole heads (a head's fp64 score matrix alone is N^2 * 8 bytes)
+ORACLE_ROWS_FROM_N = 8192
+ORACLE_SAMPLE_ROWS = 256
 METRIC = "attention TFLOP/s (bf16/fp8, causal, N=2K–16K) and % of B200 tensor peak"
 UNIT = "TFLOP/s"
 L2_FLUSH_BYTES = 256 << 20
@@ -53,8 +65,9 @@ def parse():
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
     ap.add_argument("--workload", default="attention",
-                    choices=["attention", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"],
-                    help="decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
+                    choices=["attention", "attention-2k", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"],
+                    help="attention: causal fwd+bwd, B=1 Hq=32 Hkv=8 N=16384 d=128 (default); attention-2k: causal "
+                         "fwd+bwd, B=4 Hq=Hkv=16 N=2048 d=128; decode: Nq new query rows against a KV cache (fa_fwd_kvcache), GB/s of cache read; "
                          "ring: context-parallel ring attention forward over the ranks (one GPU: 4 ranks emulated); "
                          "fp8: Hadamard-rotated e4m3 quantisation + fp8 forward (B=2 H=16 N=8192 d=128 causal); "
                          "sweep: causal fwd+bwd at N = 2K..32K with B*N = 32K tokens (H=16 d=128), plus the tiny "
@@ -66,6 +79,9 @@ def parse():
     ap.add_argument("--decode-shape", default="16,1,32,8,16384,128",
                     help="B,Nq,Hq,Hkv,Ncache,d of the decode workload")
     args = ap.parse_args()
+    if args.workload in ATTN_WORKLOADS:
+        WORKLOAD.clear()
+        WORKLOAD.update(ATTN_WORKLOADS[args.workload])
     if args.shape:
         B, Hq, Hkv, N, d, c = (int(x) for x in args.shape.split(","))
         WORKLOAD.update({"B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": bool(c),
@@ -124,10 +140,14 @@ def traffic_for(kernel, shape):
     if not os.path.exists(p) or kernel not in KERNEL_HEADER:
         return None
     j = json.load(open(p))
-    e = j.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash(kernel) or e.get("shape") != shape:
-        return None
-    return e.get("dram_bytes_per_launch")
+    entries = j.get(kernel) or []
+    if isinstance(entries, dict):
+        entries = [entries]
+    h = kernel_source_hash(kernel)
+    for e in entries:
+        if e.get("source_hash") == h and e.get("shape") == shape:
+            return e.get("dram_bytes_per_launch")
+    return None
 
 
 def step_shape(B, Hq, Hkv, N, d, causal):
@@ -226,32 +246,50 @@ def dist_setup(args):
 # ----------------------------------------------------------------- reference arm (CPU oracle)
 
 def oracle_sample(budget_s, with_bwd, w=None):
-    """Times the fp64 oracle on whole (batch, head) problems of the workload
-    (default: the bench's) until `budget_s` is spent; returns (TFLOP/s, heads
-    done, seconds, cores)."""
+    """Times the fp64 oracle on a bounded sample of the workload (default:
+    the bench's) until `budget_s` is spent: whole (batch, head) problems, or
+    for N >= ORACLE_ROWS_FROM_N the seeded 256 query rows of one (batch,
+    head) at a time (forward, and the rows' backward: their dQ and their
+    share of dK, dV). Returns (TFLOP/s, units done, seconds, cores, what a
+    unit is); flops are the algorithmic ones of the rows computed (causal:
+    row i sees i + 1 keys)."""
     import numpy as np
     import oracle
     import synth
     w = w or WORKLOAD
     q, k, v, do = synth.qkv_bf16(0, w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], with_dout=True)
     scale = 1.0 / math.sqrt(w["d"])
-    per_head = fwd_flops(1, 1, w["N"], w["d"], w["causal"]) * (3.5 if with_bwd else 1.0)
-    done, t0 = 0, time.perf_counter()
+    mult = 3.5 if with_bwd else 1.0
+    N, d = w["N"], w["d"]
+    by_rows = N >= ORACLE_ROWS_FROM_N
+    rows_all = synth.sample_rows(2, N, w["Hq"], R=ORACLE_SAMPLE_ROWS) if by_rows else None
+    done, flops, t0 = 0, 0.0, time.perf_counter()
     total = w["B"] * w["Hq"]
     while done < total:
         b, h = divmod(done, w["Hq"])
         g = oracle.kv_head_of(h, w["Hq"], w["Hkv"])
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
         slk = (slice(b, b + 1), slice(None), slice(g, g + 1))
-        oracle.attn_fwd(q[sl], k[slk], v[slk], w["causal"], scale)
-        if with_bwd:
-            oracle.attn_bwd(q[sl], k[slk], v[slk], do[sl], w["causal"], scale)
+        if by_rows:
+            r = rows_all[h:h + 1]
+            oracle.attn_fwd_rows(q[sl], k[slk], v[slk], w["causal"], scale, r)
+            if with_bwd:
+                oracle.attn_bwd_rows(q[sl], k[slk], v[slk], do[sl], w["causal"], scale, r)
+            seen = (r[0] + 1).sum() if w["causal"] else r.shape[1] * N
+            flops += 4.0 * d * float(seen) * mult
+        else:
+            oracle.attn_fwd(q[sl], k[slk], v[slk], w["causal"], scale)
+            if with_bwd:
+                oracle.attn_bwd(q[sl], k[slk], v[slk], do[sl], w["causal"], scale)
+            flops += fwd_flops(1, 1, N, d, w["causal"]) * mult
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     el = time.perf_counter() - t0
     cores = oracle_threads()[0]
-    return per_head * done / el / 1e12, done, el, cores
+    unit = (f"{ORACLE_SAMPLE_ROWS} seeded query rows of one (batch, head)" if by_rows
+            else "one whole (batch, head) problem")
+    return flops / el / 1e12, done, el, cores, unit
 
 
 def run_reference(args):
@@ -263,14 +301,15 @@ def run_reference(args):
     per_step_budget = max(0.5, min(args.cpu_budget_s, 120.0 / max(1, args.steps + args.warmup)))
     vals = []
     for i in range(args.warmup + args.steps):
-        tf, heads, el, cores = oracle_sample(per_step_budget, with_bwd)
+        tf, heads, el, cores, unit = oracle_sample(per_step_budget, with_bwd)
         if i >= args.warmup:
             vals.append((tf, heads, el))
     tf = sum(v[0] for v in vals) / len(vals)
     ms = sum(v[2] for v in vals) / len(vals) * 1e3
     heads = vals[-1][1]
     total = WORKLOAD["B"] * WORKLOAD["Hq"]
-    sample = f"{heads} of {total} (batch, head) problems per step, fp64 numpy, {'fwd+bwd' if with_bwd else 'fwd'}"
+    sample = (f"{heads} units per step (unit: {unit}; {total} (batch, head) problems in the workload), "
+              f"fp64 numpy, {'fwd+bwd' if with_bwd else 'fwd'}")
     line = {"metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -398,6 +437,12 @@ def run_ours(args):
             kk["achieved_gbs"] = kk["bytes"] / (kk["ms"] * 1e-3) / 1e9
             kk["frac"] = kk["achieved_gbs"] / pk["hbm_gbs"]
     dom = max(kernels, key=lambda x: x["ms"])
+    # the forward kernel's own roofline beside the dominant kernel's
+    fk = kernels[0]
+    forward = {"kernel": fk["kernel"], "bound": "tensor", "ms": fk["ms"], "achieved": fk["achieved_tflops"],
+               "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": fk["frac"],
+               "traffic": traffic_for(fk["kernel"], step_shape(B, Hq, Hkv, N, d, causal)),
+               "peak_source": f"{pk['source']} bf16 burst (cuBLAS)"}
     if dom["bound"] == "tensor":
         roofline = {"bound": "tensor", "kernel": dom["kernel"], "achieved": dom["achieved_tflops"],
                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": dom["frac"],
@@ -443,10 +488,10 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1:
-        tf, heads, el, cores = oracle_sample(args.cpu_budget_s, with_bwd)
+        tf, heads, el, cores, unit = oracle_sample(args.cpu_budget_s, with_bwd)
         cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
-               "sample": f"{heads} of {B * Hq} (batch, head) problems of the workload, fp64 numpy, "
-                         f"{'fwd+bwd' if with_bwd else 'fwd'}, {el:.1f} s"}
+               "sample": f"{heads} units (unit: {unit}) of the workload's {B * Hq} (batch, head) problems, "
+                         f"fp64 numpy, {'fwd+bwd' if with_bwd else 'fwd'}, {el:.1f} s"}
 
     clocks = clk.summary()
     if pg:
@@ -461,7 +506,7 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "roofline": roofline, "forward_roofline": forward, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps if with_bwd else args.steps,
             "pct_of_peak": value / world / pk["bf16_tflops"]}
     print(json.dumps(line), flush=True)
@@ -1450,7 +1495,7 @@ def run_sweep(args):
     value = tot_flops * world / (tot_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1:
-        tf, heads, el, cores = oracle_sample(args.cpu_budget_s, True, sweep_workload(SWEEP_NS[0]))
+        tf, heads, el, cores, _ = oracle_sample(args.cpu_budget_s, True, sweep_workload(SWEEP_NS[0]))
         cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "blas": oracle_threads()[1],
                "sample": f"{heads} (batch, head) problems of the N=2048 point, fp64 numpy, fwd+bwd, {el:.1f} s"}
     clocks = clk.summary()

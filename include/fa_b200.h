@@ -55,7 +55,9 @@ typedef enum {
 } fa_status_t;
 
 /*
- * Forward pass, padded batch.
+ * Forward pass, padded batch (the exact tiled attention of the catalogue
+ * record "Dao and colleagues: IO-aware exact attention with FlashAttention",
+ * field summary).
  *   q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 (in);  o [B,N,Hq,d] bf16 (out);
  *   lse [B,Hq,N] float32 (out, natural log of the scaled scores' row sums).
  *   causal: 0 or 1 (query i sees keys 0..i).  scale: > 0 and finite, usually 1/sqrt(d).
@@ -97,7 +99,8 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
                        int N, int d, int causal, float scale, void* stream);
 
 /*
- * Bytes of device workspace fa_bwd / fa_bwd_varlen need: two fp32 vectors per
+ * Bytes of device workspace fa_bwd / fa_bwd_varlen need (the statistics the
+ * recomputing backward of the catalogue record's summary reads back): two fp32 vectors per
  * (query head, token), the row's LSE in base 2 and D = dot(dO, O); each
  * sequence's rows start 16-byte aligned, plus 128 padding rows per head.
  * tokens = B*N (padded) or total_T (varlen); nseq = B or the number of packed
@@ -106,7 +109,15 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
 
 /*
- * Backward pass, padded batch: gradients of sum(O * dout) with respect to
+ * The smallest workspace fa_bwd / fa_bwd_varlen accept (same arguments as
+ * fa_bwd_workspace_size): the two fp32 vectors per (query head, token) alone.
+ */
+size_t fa_bwd_min_workspace_size(int tokens, int nseq, int Hq, int d);
+
+/*
+ * Backward pass, padded batch (the catalogue record's summary: recomputation
+ * instead of a stored attention matrix; the Dao-AILab repository overview:
+ * deterministic backward): gradients of sum(O * dout) with respect to
  * q, k, v, recomputing the scores from q, k, v and the forward's lse.
  *   q, k, v, o, dout bf16, lse f32 (in, as produced by fa_fwd);
  *   dq [B,N,Hq,d], dk/dv [B,N,Hkv,d] bf16 (out; dk/dv summed over the query
@@ -145,24 +156,32 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
  * convenience.)
  *   Arguments and results as fa_bwd, minus the workspace: the scratch lives in
  *   an 8 MiB array inside the library, on every device that loads it, for the
- *   life of the process. The problem must fit it:
- *   fa_bwd_workspace_size(B*N, B, Hq, d) <= 8 MiB, i.e. Hq * (B*N + 4*B + 131)
- *   up to about 1.04 million; larger problems return FA_ERR_WORKSPACE and launch
- *   nothing.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   life of the process. It runs exactly what fa_bwd runs with a workspace of
+ *   fa_bwd_min_workspace_size bytes (bitwise the same results). The problem
+ *   must fit the array: fa_bwd_min_workspace_size(B*N, B, Hq, d) <= 8 MiB,
+ *   i.e. Hq * (B*N + 4*B + 131) up to about 1.04 million; larger problems
+ *   return FA_ERR_WORKSPACE and launch nothing.
+ *   Set-up on the first call on each device, with that device current: the
+ *   array's device address is looked up (cudaGetSymbolAddress), and, as for
+ *   the first fa_bwd on a device, a second stream and two events are created
+ *   (the dQ kernel runs on that stream beside the dK/dV kernel). Make that
+ *   first call before any stream capture.
  *   Every call uses the same array: calls whose work overlaps on the GPU (on
  *   different streams, or from different threads) race on it and must be
  *   serialised by the caller. The array keeps whatever the last call left;
  *   nothing in it needs clearing between calls.
  *   No cudaMalloc, cudaFree or other allocating routine is called.
+ *   The library caches per-device state (these addresses, the stream and the
+ *   events) for the life of the process: cudaDeviceReset while it is loaded
+ *   is not supported.
  */
 fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                            const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
                            int causal, float scale, void* stream);
 
-/* Backward pass, packed variable-length batch; layouts as fa_fwd_varlen. */
+/* Backward pass, packed variable-length batch (the varlen API of the
+ * Dao-AILab repository overview; recomputation as fa_bwd); layouts as
+ * fa_fwd_varlen. */
 fa_status_t fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                           const int* cu_seqlens, int nseq, int max_seqlen, int total_T, int Hq, int Hkv, int d,

@@ -587,10 +587,14 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
   return launch_fwd<128, 0, true>(ds, q8, k8, v8, a, B * N, bound, static_cast<cudaStream_t>(stream));
 }
 
-size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
+size_t fa_bwd_min_workspace_size(int tokens, int nseq, int Hq, int d) {
   (void)d;
   if (tokens <= 0 || Hq <= 0 || nseq < 0) return 0;
   return 2 * vec_bytes(tokens, nseq, Hq);
+}
+
+size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
+  return fa_bwd_min_workspace_size(tokens, nseq, Hq, d);
 }
 
 size_t fa_bwd_blocksparse_workspace_size(int B, int Hq, int Hkv, int N, int d) {
@@ -651,15 +655,15 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   if (B < 0 || N < 0 || Hq <= 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * N == 0) return FA_OK;
   if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
-  // the whole working set must fit the built-in array
-  if (fa_bwd_workspace_size(B * N, B, Hq, d) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  // the whole working set (the two-vector workspace) must fit the built-in array
+  const size_t need = fa_bwd_min_workspace_size(B * N, B, Hq, d);
+  if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const fa_status_t st = noalloc_scratch_address(&scratch);
   if (st != FA_OK) return st;
   // Nothing in the scratch has to start at zero: the first kernel of the
   // backward writes every entry the later two read.
-  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, kNoAllocScratchBytes, B, Hq, Hkv, N, d, causal, scale,
-                stream);
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, need, B, Hq, Hkv, N, d, causal, scale, stream);
 }
 
 size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Hq, int d, int num_splits) {

@@ -16,7 +16,7 @@ BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_ste
              "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
 
 
-@pytest.mark.parametrize("workload", ["attention", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"])
+@pytest.mark.parametrize("workload", ["attention", "attention-2k", "decode", "ring", "fp8", "blocksparse", "sweep", "varlen"])
 def test_reference_arm_prints_one_contract_line(workload):
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
                           workload, "--steps", "1", "--warmup", "0", "--cpu-budget-s", "0.3"],
@@ -37,13 +37,16 @@ def test_reference_arm_prints_one_contract_line(workload):
 def test_traffic_lookup_is_keyed_by_shape():
     import bench
     j = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
-    for kernel, e in j.items():
+    for kernel, entries in j.items():
         if kernel.startswith("_"):
             continue
-        assert isinstance(e["shape"], str) and e["dram_bytes_per_launch"] > 0
-        if e["source_hash"] == bench.kernel_source_hash(kernel):
-            assert bench.traffic_for(kernel, e["shape"]) == e["dram_bytes_per_launch"]
-        assert bench.traffic_for(kernel, e["shape"] + " other") is None
+        shapes = [e["shape"] for e in entries]
+        assert len(shapes) == len(set(shapes)), kernel
+        for e in entries:
+            assert isinstance(e["shape"], str) and e["dram_bytes_per_launch"] > 0
+            if e["source_hash"] == bench.kernel_source_hash(kernel):
+                assert bench.traffic_for(kernel, e["shape"]) == e["dram_bytes_per_launch"]
+            assert bench.traffic_for(kernel, e["shape"] + " other") is None
 
 
 def _max_rank_main(rank, world, port, q):

@@ -84,9 +84,10 @@ def test_bwd_varlen_small(fa, causal):
     _check_grads((dq, dk, dv), want, "varlen small bwd")
 
 
-def test_config_varlen_fwd_bwd(fa):
-    """Varlen packed causal forward + backward: 24 sequences, lengths U[128,4096]
-    (seed 0), H=16, d=128; O/LSE and all gradients checked on 4 of the 16 heads."""
+@pytest.fixture(scope="module")
+def varlen_cfg(fa):
+    """The packed causal workload: 24 sequences, lengths U[128,4096] (seed 0),
+    H=16, d=128; inputs and the GPU forward + backward, computed once."""
     lengths = synth.varlen_lengths(0)
     H, d = 16, 128
     q, k, v, do, cu = synth.qkv_varlen_bf16(0, lengths, H, H, d, with_dout=True)
@@ -98,13 +99,64 @@ def test_config_varlen_fwd_bwd(fa):
     dq, dk, dv = fa.attention_bwd_varlen(qd, kd, vd, o, lse, dod, cu_d, mx, causal=True)
     torch.cuda.synchronize()
     assert fa.fa_get_status() == fa.FA_OK
-    heads = [0, 7, 15]
+    return (q, k, v, do, cu), tuple(t.cpu() for t in (o, lse, dq, dk, dv))
+
+
+@pytest.mark.parametrize("heads", [[0, 1, 2, 3], [4, 5, 6, 7], [8, 9, 10, 11], [12, 13, 14, 15]])
+def test_config_varlen_fwd_bwd(varlen_cfg, heads):
+    """Varlen packed causal forward + backward, every sequence: O, LSE and all
+    gradients against the oracle, four of the 16 heads per case (all 16
+    over the four cases)."""
+    (q, k, v, do, cu), (o, lse, dq, dk, dv) = varlen_cfg
+    d = q.shape[2]
     sl = (slice(None), heads)
     want = oracle.attn_bwd_varlen(q[sl], k[sl], v[sl], do[sl], cu, True, 1 / math.sqrt(d))
-    _check_grads((dq[sl], dk[sl], dv[sl]), want, "cfg5 bwd")
+    _check_grads((dq[sl], dk[sl], dv[sl]), want, f"cfg5 bwd heads {heads}")
     O, L = oracle.attn_fwd_varlen(q[sl], k[sl], v[sl], cu, True, 1 / math.sqrt(d))
-    assert oracle.rel_rms(o[sl].cpu(), O) <= 5e-3
-    assert float(np.max(np.abs(lse[heads].cpu().double().numpy() - L))) <= 1e-3
+    assert oracle.rel_rms(o[sl], O) <= 5e-3
+    assert oracle.max_abs(o[sl], O) <= 2e-2
+    assert float(np.max(np.abs(lse[heads].double().numpy() - L))) <= 1e-3
+
+
+def test_bwd_config_long_context_gqa(fa):
+    """Backward of the long-context GQA workload (B=1, Hq=32, Hkv=8, N=16384,
+    d=128, causal; the bench's default launch): dQ on 64 seeded query rows of
+    every head against the oracle's row-sampled backward, and dK, dV of three
+    key tiles of kv head 3 against the oracle's key-block gradient given the
+    oracle's own O and LSE of every row of that head's four query heads."""
+    B, N, Hq, Hkv, d = 1, 16384, 32, 8, 128
+    scale = 1 / math.sqrt(d)
+    q, k, v, do = synth.qkv_bf16(0, B, N, Hq, Hkv, d, with_dout=True)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    o, lse = fa.attention_fwd(qd, kd, vd, causal=True, scale=scale)
+    dq, dk, dv = fa.attention_bwd(qd, kd, vd, o, lse, dod, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
+    rows = synth.sample_rows(2, N, Hq, R=64)
+    wq, _, _ = oracle.attn_bwd_rows(q, k, v, do, True, scale, rows)
+    gq = np.stack([dq[0, rows[h], h].double().numpy() for h in range(Hq)])
+    assert np.all(np.isfinite(gq))
+    assert oracle.rel_rms(gq, wq[0]) <= G_REL_RMS
+    g = 3
+    heads = list(range(g * (Hq // Hkv), (g + 1) * (Hq // Hkv)))
+    qh, doh = q[:, :, heads], do[:, :, heads]
+    kh, vh = k[:, :, g:g + 1], v[:, :, g:g + 1]
+    allrows = np.tile(np.arange(N), (len(heads), 1))
+    O = np.empty((B, N, len(heads), d))
+    L = np.empty((B, len(heads), N))
+    for c in range(0, N, 2048):  # the oracle forward of every row, in row chunks
+        Oc, Lc = oracle.attn_fwd_rows(qh, kh, vh, True, scale, allrows[:, c:c + 2048])
+        O[:, c:c + 2048] = Oc.transpose(0, 2, 1, 3)
+        L[:, :, c:c + 2048] = Lc
+    for kb in (0, 61, 127):
+        j0 = kb * 128
+        _, wk, wv = oracle.attn_bwd_block(qh[:, j0:], kh[:, j0:j0 + 128], vh[:, j0:j0 + 128], doh[:, j0:],
+                                          O[:, j0:], L[:, :, j0:], True, scale)
+        for name, got, want in (("dk", dk[:, j0:j0 + 128, g:g + 1], wk), ("dv", dv[:, j0:j0 + 128, g:g + 1], wv)):
+            rr = oracle.rel_rms(got.double().numpy(), want)
+            assert rr <= G_REL_RMS, f"key tile {kb} {name} rel-RMS {rr}"
 
 
 def test_bwd_deterministic(fa):
