@@ -109,12 +109,6 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d);
 
 /*
- * The smallest workspace fa_bwd / fa_bwd_varlen accept (same arguments as
- * fa_bwd_workspace_size): the two fp32 vectors per (query head, token) alone.
- */
-size_t fa_bwd_min_workspace_size(int tokens, int nseq, int Hq, int d);
-
-/*
  * Backward pass, padded batch (the catalogue record's summary: recomputation
  * instead of a stored attention matrix; the Dao-AILab repository overview:
  * deterministic backward): gradients of sum(O * dout) with respect to
@@ -156,9 +150,9 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
  * convenience.)
  *   Arguments and results as fa_bwd, minus the workspace: the scratch lives in
  *   an 8 MiB array inside the library, on every device that loads it, for the
- *   life of the process. It runs exactly what fa_bwd runs with a workspace of
- *   fa_bwd_min_workspace_size bytes (bitwise the same results). The problem
- *   must fit the array: fa_bwd_min_workspace_size(B*N, B, Hq, d) <= 8 MiB,
+ *   life of the process. It runs exactly what fa_bwd runs (bitwise the same
+ *   results). The problem must fit the array:
+ *   fa_bwd_workspace_size(B*N, B, Hq, d) <= 8 MiB,
  *   i.e. Hq * (B*N + 4*B + 131) up to about 1.04 million; larger problems
  *   return FA_ERR_WORKSPACE and launch nothing.
  *   Set-up on the first call on each device, with that device current: the

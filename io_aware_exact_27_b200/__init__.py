@@ -58,8 +58,6 @@ for _name, _args in _SIGS.items():
     getattr(_lib, _name).restype = _I
 _lib.fa_bwd_workspace_size.argtypes = [_I, _I, _I, _I]
 _lib.fa_bwd_workspace_size.restype = _Z
-_lib.fa_bwd_min_workspace_size.argtypes = [_I, _I, _I, _I]
-_lib.fa_bwd_min_workspace_size.restype = _Z
 _lib.fa_bwd_blocksparse_workspace_size.argtypes = [_I, _I, _I, _I, _I]
 _lib.fa_bwd_blocksparse_workspace_size.restype = _Z
 _lib.fa_fwd_kvcache_workspace_size.argtypes = [_I, _I, _I, _I, _I]
@@ -130,10 +128,6 @@ def fa_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, Hq, Hkv, N, d, 
 
 def fa_bwd_workspace_size(tokens, nseq, Hq, d) -> int:
     return int(_lib.fa_bwd_workspace_size(tokens, nseq, Hq, d))
-
-
-def fa_bwd_min_workspace_size(tokens, nseq, Hq, d) -> int:
-    return int(_lib.fa_bwd_min_workspace_size(tokens, nseq, Hq, d))
 
 
 def fa_bwd_blocksparse_workspace_size(B, Hq, Hkv, N, d) -> int:

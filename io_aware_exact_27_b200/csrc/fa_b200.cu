@@ -587,14 +587,10 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
   return launch_fwd<128, 0, true>(ds, q8, k8, v8, a, B * N, bound, static_cast<cudaStream_t>(stream));
 }
 
-size_t fa_bwd_min_workspace_size(int tokens, int nseq, int Hq, int d) {
+size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
   (void)d;
   if (tokens <= 0 || Hq <= 0 || nseq < 0) return 0;
   return 2 * vec_bytes(tokens, nseq, Hq);
-}
-
-size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
-  return fa_bwd_min_workspace_size(tokens, nseq, Hq, d);
 }
 
 size_t fa_bwd_blocksparse_workspace_size(int B, int Hq, int Hkv, int N, int d) {
@@ -655,8 +651,8 @@ fa_status_t fa_bwd_noalloc(const void* q, const void* k, const void* v, const vo
   if (B < 0 || N < 0 || Hq <= 0) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * N == 0) return FA_OK;
   if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
-  // the whole working set (the two-vector workspace) must fit the built-in array
-  const size_t need = fa_bwd_min_workspace_size(B * N, B, Hq, d);
+  // the whole working set must fit the built-in array
+  const size_t need = fa_bwd_workspace_size(B * N, B, Hq, d);
   if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const fa_status_t st = noalloc_scratch_address(&scratch);

@@ -120,18 +120,18 @@ def test_torch_wrappers_reject_what_the_library_cannot_read():
 
 def test_noalloc_size_limit_on_the_host(lib):
     """fa_bwd_noalloc's size check runs before any device call: a problem
-    whose two-vector workspace exceeds the 8 MiB array is refused with
+    whose workspace (fa_bwd_workspace_size) exceeds the 8 MiB array is refused with
     FA_ERR_WORKSPACE; one that just fits passes the check and then stops
     at a later host-side check (null tensors), launching nothing."""
     P, I = ctypes.c_void_p, ctypes.c_int
     lib.fa_bwd_noalloc.argtypes = [P] * 9 + [I] * 6 + [ctypes.c_float, P]
-    lib.fa_bwd_min_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     fake = P(256)
     limit = 8 << 20
     H, d = 16, 128
     # largest N (B = 1) whose workspace fits, found from the size function itself
-    fits = max(n for n in range(60000, 70000, 4) if lib.fa_bwd_min_workspace_size(n, 1, H, d) <= limit)
-    assert lib.fa_bwd_min_workspace_size(fits + 4, 1, H, d) > limit
+    fits = max(n for n in range(60000, 70000, 4) if lib.fa_bwd_workspace_size(n, 1, H, d) <= limit)
+    assert lib.fa_bwd_workspace_size(fits + 4, 1, H, d) > limit
     assert lib.fa_bwd_noalloc(*([fake] * 9), 1, H, H, fits + 4, d, 1, 0.1, None) == 5
     # null tensors: past the size check the call stops at the device lookup
     # (no GPU) or at the pointer checks (GPU): nothing is launched either way

@@ -159,6 +159,23 @@ def test_bwd_config_long_context_gqa(fa):
             assert rr <= G_REL_RMS, f"key tile {kb} {name} rel-RMS {rr}"
 
 
+def test_bwd_deterministic_gqa_long(fa):
+    """GQA, long causal sequence, dK/dV and dQ kernels running side by side
+    on two streams: every output element still has one writer and a fixed
+    summation order, so repeated runs agree bitwise."""
+    q, k, v, do = synth.qkv_bf16(29, 1, 4096, 16, 4, 128, with_dout=True)
+    dev = torch.device("cuda")
+    q, k, v, do = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    o, lse = fa.attention_fwd(q, k, v, causal=True)
+    g1 = fa.attention_bwd(q, k, v, o, lse, do, causal=True)
+    for _ in range(3):
+        g2 = fa.attention_bwd(q, k, v, o, lse, do, causal=True)
+        torch.cuda.synchronize()
+        assert fa.fa_get_status() == fa.FA_OK
+        for a, b in zip(g1, g2):
+            assert torch.equal(a, b)
+
+
 def test_bwd_deterministic(fa):
     """The reduction order of every gradient is fixed: two runs agree bitwise."""
     q, k, v, do = synth.qkv_bf16(23, 2, 1024, 8, 2, 128, with_dout=True)

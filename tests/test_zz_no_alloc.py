@@ -36,10 +36,9 @@ def _case(fa, B, N, Hq, Hkv, d, causal, seed):
     q, k, v, do = q_h.to(dev), k_h.to(dev), v_h.to(dev), do_h.to(dev)
     scale = 1 / math.sqrt(d)
     o, lse = fa.attention_fwd(q, k, v, causal=causal, scale=scale)
-    # fa_bwd on a caller-provided workspace of the size the no-allocation
-    # call runs with (the two-vector workspace): the same kernels, so the
+    # fa_bwd on a caller-provided workspace: the same kernels, so the
     # results must be bitwise equal
-    ws_bytes = fa.fa_bwd_min_workspace_size(B * N, B, Hq, d)
+    ws_bytes = fa.fa_bwd_workspace_size(B * N, B, Hq, d)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     want = tuple(torch.empty_like(t) for t in (q, k, v))
     fa.fa_bwd(q, k, v, o, lse, do, *want, ws, ws_bytes, B, Hq, Hkv, N, d, int(causal), scale)
@@ -61,8 +60,8 @@ def test_noalloc_matches_fa_bwd_twice(fa):
 
 
 def test_noalloc_rejects_oversized_problem(fa):
-    # the two-vector workspace (about Hq * (B*N + 131) * 8 bytes) beyond the
-    # 8 MiB array: rejected before any launch
+    # the workspace (about Hq * (B*N + 131) * 8 bytes) beyond the 8 MiB
+    # array: rejected before any launch
     B, N, H, d = 1, 70000, 16, 128
     with pytest.raises(fa.FAError) as e:
         fa.fa_bwd_noalloc(16, 16, 16, 16, 16, 16, 16, 16, 16, B, H, H, N, d, 1, 0.1)
