@@ -355,16 +355,6 @@ void fa_set_wait_timeout_ns(uint64_t ns);
  */
 void fa_debug_set_inject(int mode);
 
-/*
- * Tuning knob of the bf16 forward kernels (the fp8 forward always uses
- * MUFU): of every 8 pairs of score
- * elements, how many take their exponential on the FMA pipe (a cubic
- * polynomial after exact range reduction, relative error < 1e-4) instead of
- * the MUFU unit. Accepted: 0, 2, 3 (default 0, the fastest measured); other
- * values return FA_ERR_UNSUPPORTED. Blocks that contain masked keys always use
- * MUFU. Affects launches made after the call.
- */
-fa_status_t fa_set_exp_emulation(int pairs_of_8);
 
 #ifdef __cplusplus
 }

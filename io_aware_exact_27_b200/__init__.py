@@ -42,7 +42,6 @@ _SIGS = {
     "fa_bwd": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_varlen": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_get_status": [_P],
-    "fa_set_exp_emulation": [_I],
     "fa_fwd_kvcache": [_P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P],
     "fa_attn_merge": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P],
     "fa_fp8_quantize": [_P, _P, _P, _I, _I, _I, _I, _I, _P],
@@ -289,10 +288,6 @@ def fa_last_device_error_word() -> int:
 
 def fa_set_wait_timeout_ns(ns: int):
     _lib.fa_set_wait_timeout_ns(int(ns))
-
-
-def fa_set_exp_emulation(pairs_of_8: int):
-    _check(_lib.fa_set_exp_emulation(int(pairs_of_8)), "fa_set_exp_emulation")
 
 
 def fa_debug_set_inject(mode: int):

@@ -27,7 +27,6 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 
 std::atomic<uint64_t> g_timeout_ns{4000000000ull};
 std::atomic<int> g_inject{0};
-std::atomic<int> g_exp_emu{0};  // pairs of every 8 whose exp2 runs on the FMA pipe
 std::atomic<int> g_last_word{0};
 
 constexpr int kMaxDevices = 64;
@@ -37,7 +36,7 @@ struct DeviceState {
   int sms = 0;
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
-  bool fwd_attr[3][6][2] = {};  // [bf16 d64, bf16 d128, fp8][EMU][block-sparse]
+  bool fwd_attr[3][2] = {};  // [bf16 d64, bf16 d128, fp8][block-sparse]
   bool bwd_attr[2][2] = {{false, false}, {false, false}};  // [d == 128][block-sparse]
   bool dec_attr[2] = {false, false};
   // the backward runs its dQ kernel beside the dK/dV kernel: a second stream
@@ -114,16 +113,16 @@ fa_status_t check_common(const void* q, const void* k, const void* v, const void
   return FA_OK;
 }
 
-template <int D, int EMU, bool F8 = false, bool SPARSE = false>
+template <int D, bool F8 = false, bool SPARSE = false>
 fa_status_t launch_fwd(DeviceState* ds, const void* q, const void* k, const void* v, fa::FwdArgs a, int tokens,
                        long long units_bound, cudaStream_t stream) {
   constexpr int STAGES = F8 ? 6 : 4;
   using Smem = fa::FwdSmem<D, STAGES, F8>;
-  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, EMU, F8, SPARSE>;
+  auto kern = fa::fa_fwd_sm100_kernel<D, STAGES, F8, SPARSE>;
   const int smem = static_cast<int>(sizeof(Smem)) + 1024;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->fwd_attr[F8 ? 2 : (D == 128 ? 1 : 0)][EMU][SPARSE ? 1 : 0];
+    bool& done = ds->fwd_attr[F8 ? 2 : (D == 128 ? 1 : 0)][SPARSE ? 1 : 0];
     if (!done) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return FA_ERR_CUDA;
@@ -183,18 +182,11 @@ fa_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, f
   }
   if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (block_mask != nullptr)  // block-sparse: MUFU exponentials only
-    return d == 128 ? launch_fwd<128, 0, false, true>(ds, q, k, v, a, total_T, bound, s)
-                    : launch_fwd<64, 0, false, true>(ds, q, k, v, a, total_T, bound, s);
-  switch ((d == 128 ? 10 : 0) + g_exp_emu.load()) {
-    case 0: return launch_fwd<64, 0>(ds, q, k, v, a, total_T, bound, s);
-    case 2: return launch_fwd<64, 2>(ds, q, k, v, a, total_T, bound, s);
-    case 3: return launch_fwd<64, 3>(ds, q, k, v, a, total_T, bound, s);
-    case 10: return launch_fwd<128, 0>(ds, q, k, v, a, total_T, bound, s);
-    case 12: return launch_fwd<128, 2>(ds, q, k, v, a, total_T, bound, s);
-    case 13: return launch_fwd<128, 3>(ds, q, k, v, a, total_T, bound, s);
-  }
-  return FA_ERR_UNSUPPORTED;
+  if (block_mask != nullptr)
+    return d == 128 ? launch_fwd<128, false, true>(ds, q, k, v, a, total_T, bound, s)
+                    : launch_fwd<64, false, true>(ds, q, k, v, a, total_T, bound, s);
+  return d == 128 ? launch_fwd<128>(ds, q, k, v, a, total_T, bound, s)
+                  : launch_fwd<64>(ds, q, k, v, a, total_T, bound, s);
 }
 
 // Floats per head of each backward workspace vector (see fa::ws_offset).
@@ -584,7 +576,7 @@ fa_status_t fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const flo
   if (bound > INT32_MAX) return FA_ERR_UNSUPPORTED;
   a.num_units = static_cast<int>(bound);
   // exponentials on MUFU only: the FMA pipe is shared with the V widening warps
-  return launch_fwd<128, 0, true>(ds, q8, k8, v8, a, B * N, bound, static_cast<cudaStream_t>(stream));
+  return launch_fwd<128, true>(ds, q8, k8, v8, a, B * N, bound, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int tokens, int nseq, int Hq, int d) {
@@ -872,11 +864,5 @@ const char* fa_status_string(fa_status_t s) {
 void fa_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 1 : ns); }
 
 void fa_debug_set_inject(int mode) { g_inject.store(mode); }
-
-fa_status_t fa_set_exp_emulation(int pairs_of_8) {
-  if (pairs_of_8 != 0 && pairs_of_8 != 2 && pairs_of_8 != 3) return FA_ERR_UNSUPPORTED;
-  g_exp_emu.store(pairs_of_8);
-  return FA_OK;
-}
 
 }  // extern "C"

@@ -223,9 +223,9 @@ __device__ __forceinline__ bool warp_tile_on(const WarpMaskRows& w, int tile, in
 
 // Exponentials of 2*NP consecutive columns of one row: p = 2^(s*cj - m),
 // packed in pairs (bf16, or f16 of p*pmul on the fp8 path) into pk[NP] for
-// the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs;
-// EMU of every 8 pairs take exp2 on the FMA pipe (exp2_poly_pair).
-template <int EMU, bool F16, int NP = 32>
+// the PV MMA; returns the fp32 sum. Scale and sum run on packed fp32 pairs,
+// the exponentials on the MUFU unit.
+template <bool F16, int NP = 32>
 __device__ __forceinline__ float exp_pack(const float* s, float cj, float m, float pmul, uint32_t* pk) {
   const uint64_t c2 = f2(cj, cj);
   const uint64_t nm2 = f2(-m, -m);
@@ -233,14 +233,9 @@ __device__ __forceinline__ float exp_pack(const float* s, float cj, float m, flo
 #pragma unroll
   for (int t = 0; t < NP; ++t) {
     const uint64_t x2 = f2_fma(f2(s[2 * t], s[2 * t + 1]), c2, nm2);
-    float p0, p1;
-    if ((t & 7) < EMU) {
-      exp2_poly_pair(x2, p0, p1);
-    } else {
-      const float2 x = f2_split(x2);
-      p0 = ex2_approx(x.x);
-      p1 = ex2_approx(x.y);
-    }
+    const float2 x = f2_split(x2);
+    const float p0 = ex2_approx(x.x);
+    const float p1 = ex2_approx(x.y);
     acc[t & 3] = f2_add(acc[t & 3], f2(p0, p1));
     if constexpr (F16)
       pk[t] = pack_f16x2(p0 * pmul, p1 * pmul);
@@ -251,7 +246,7 @@ __device__ __forceinline__ float exp_pack(const float* s, float cj, float m, flo
   return a.x + a.y;
 }
 
-template <int D, int STAGES, int EMU, bool F8, bool SPARSE = false>
+template <int D, int STAGES, bool F8, bool SPARSE = false>
 __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const FwdArgs args) {
@@ -612,8 +607,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
           uint32_t pk[16];
           // a row that has seen no visible key yet (block-sparse) keeps
           // m = -inf: its exponentials are taken against 0 and are all 0
-          lsum += masked_blk ? exp_pack<0, F8, 16>(sv, cj, SPARSE && m_new == -INFINITY ? 0.f : m_new, pmul, pk)
-                             : exp_pack<EMU, F8, 16>(sv, cj, m_new, pmul, pk);
+          lsum += masked_blk ? exp_pack<F8, 16>(sv, cj, SPARSE && m_new == -INFINITY ? 0.f : m_new, pmul, pk)
+                             : exp_pack<F8, 16>(sv, cj, m_new, pmul, pk);
           tmem_st16(S + 16 * c, pk);
         }
         l = l * alpha + lsum;

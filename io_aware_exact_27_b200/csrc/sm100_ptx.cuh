@@ -366,32 +366,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
-// 2^x for a pair of floats on the FMA/ALU pipes instead of MUFU (x <= 127).
-// Method: Cody-Waite style split x = n + f with n = round(x) obtained by the
-// round-to-nearest addition of 1.5*2^23, f in [-0.5, 0.5]; 2^f by a cubic
-// fitted to 2^f on [-0.5, 0.5] (iteratively reweighted least squares in the
-// relative sense, max relative error 7.5e-5); 2^n added to the exponent field
-// as an integer. Inputs below -125 are clamped to -125 (2^-125 ~ 2.4e-38), so
-// the result is never denormal or wrapped.
-__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& r0, float& r1) {
-  float2 x = f2_split(x2);
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const uint64_t xc = f2(x.x, x.y);
-  const uint64_t magic = f2(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(xc, magic);
-  const uint64_t n = f2_add(t, f2(-12582912.f, -12582912.f));
-  const uint64_t fr = f2_fma(n, f2(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(fr, f2(0.05517132207751274f, 0.05517132207751274f),
-                      f2(0.24261054396629333f, 0.24261054396629333f));
-  p = f2_fma(p, fr, f2(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, fr, f2(0.9999281167984009f, 0.9999281167984009f));
-  const float2 pv = f2_split(p);
-  const float2 tv = f2_split(t);
-  r0 = __uint_as_float(__float_as_uint(pv.x) + (__float_as_uint(tv.x) << 23));
-  r1 = __uint_as_float(__float_as_uint(pv.y) + (__float_as_uint(tv.y) << 23));
-}
-
 // Four floats to four e4m3 bytes (round to nearest even, saturating), the
 // first element in the lowest byte: the order tcgen05 reads an 8-bit A
 // operand from a 32-bit TMEM column.

@@ -219,19 +219,3 @@ def test_bounded_wait_reports_timeout(fa):
     assert fa.fa_get_status() == fa.FA_OK
     O, L = oracle.attn_fwd(q.cpu(), k.cpu(), v.cpu(), False, 1 / math.sqrt(d))
     _check_o_lse(o, lse, O, L, "after timeout")
-
-
-@pytest.mark.parametrize("emu", [0, 2, 3])
-@pytest.mark.parametrize("causal", [False, True])
-def test_exp_emulation_variants(fa, emu, causal):
-    """Every accepted split of the exponentials between MUFU and the FMA-pipe
-    polynomial meets the same tolerances."""
-    fa.fa_set_exp_emulation(emu)
-    try:
-        (q, k, v), o, lse = _run_padded(fa, 2, 1024, 4, 2, 128, causal, seed=17)
-    finally:
-        fa.fa_set_exp_emulation(0)
-    O, L = oracle.attn_fwd(q, k, v, causal, 1 / math.sqrt(128))
-    _check_o_lse(o, lse, O, L, f"emu={emu}")
-    with pytest.raises(fa.FAError):
-        fa.fa_set_exp_emulation(1)
