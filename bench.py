@@ -1059,7 +1059,8 @@ def run_fp8(args):
     ach = flops / (f_ms * 1e-3) / 1e12
     q_bytes = 3 * B * N * H * d * (2 + 1) + 3 * B * H * nblk * 4
     roofline = {"bound": "tensor", "kernel": "fa_fwd_sm100_kernel (fp8)", "achieved": ach, "peak": fp8_peak,
-                "unit": "TFLOP/s", "frac": ach / fp8_peak, "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / fp8_peak,
+                "traffic": traffic_for("fa_fwd_sm100_kernel", "fp8 " + step_shape(B, H, H, N, d, True)),
                 "peak_source": f"{pk['source']} bf16 burst x 2 (nominal e4m3/bf16 ratio)",
                 "note": "S = Q K^T runs at the e4m3 rate, O += P V at the 16-bit rate (P and V as f16): "
                         "at most 4/3 of the bf16 peak for this kernel",
