@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   const uint32_t tmem = sm.tmem_base;
   // TMEM: S0 [0,128) S1 [128,256) dP [256,384) dQ [384, 384+D)
   const uint32_t tS0 = tmem, tDP = tmem + 256, tDQ = tmem + 384;
-  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 7};
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 7,
+                 !SPARSE && !varlen && !args.causal};
   const volatile int* abort = &sm.abort;
   const int group = args.Hq / args.Hkv;
   uint32_t prod_issued = 0, q_issued = 0;
@@ -435,7 +436,8 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   // TMEM: S^T [0,128) dP^T [128,256) dV [256,256+D) dK [384,384+D)
   const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
   // causal: the heaviest key tiles are the first ones (most query tiles see them)
-  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hkv, args.causal, nlevels, sm.level_count, 7};
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hkv, args.causal, nlevels, sm.level_count, 7,
+                 !SPARSE && !varlen && !args.causal};
   const volatile int* abort = &sm.abort;
   const int group = args.Hq / args.Hkv;
   uint32_t prod_issued = 0, kv_issued = 0;

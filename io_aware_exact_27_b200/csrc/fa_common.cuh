@@ -27,7 +27,11 @@ __device__ __forceinline__ void report_error(int* status, int code, int site) {
 // the sequence; `ascending` walks the levels from tile 0 upwards, otherwise
 // from the last tile down, so that for causal attention the heaviest units
 // come first. Heads vary fastest, so concurrently running units of one GQA
-// group share their K/V tiles in L2.
+// group share their K/V tiles in L2. With `level_fastest` (padded batches
+// whose units all cost the same: dense, non-causal) the levels vary fastest
+// instead: the units running at one time then cover a few (sequence, head)
+// pairs whole, and their K/V working set stays in L2 however many pairs the
+// batch has.
 struct SeqSched {
   const int* cu_seqlens;  // varlen: device [nseq+1]; padded: nullptr
   int nseq;               // padded: B
@@ -37,6 +41,7 @@ struct SeqSched {
   int nlevels;            // ceil(N >> shift)
   const int* level_count; // varlen: smem [nlevels], sequences holding > L units
   int shift;              // log2 of the rows of a unit
+  int level_fastest;      // padded only: unit u = pair * nlevels + level (see above)
 };
 
 struct Unit {
@@ -51,8 +56,8 @@ __device__ __forceinline__ Unit decode_unit(const SeqSched& s, int u) {
   Unit r;
   if (s.cu_seqlens == nullptr) {
     const int BH = s.nseq * s.heads;
-    const int level = u / BH;
-    const int rem = u - level * BH;
+    const int level = s.level_fastest ? u % s.nlevels : u / BH;
+    const int rem = s.level_fastest ? u / s.nlevels : u - level * BH;
     r.qb2 = s.ascending ? level : (s.nlevels - 1 - level);
     r.h = rem % s.heads;
     r.seq = rem / s.heads;

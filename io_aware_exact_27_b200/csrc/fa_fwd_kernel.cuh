@@ -303,7 +303,8 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
     num_units = varlen_level_table(sm.level_count, args.cu_seqlens, args.nseq, nlevels, 8, args.Hq, kThreads);
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 8};
+  SeqSched sched{args.cu_seqlens, args.nseq, args.N, args.Hq, !args.causal, nlevels, sm.level_count, 8,
+                 !SPARSE && !varlen && !args.causal};
   const volatile int* abort = &sm.abort;
   const int group = args.Hq / args.Hkv;
   uint32_t prod_issued = 0;  // K/V loads issued by the producer thread
