@@ -221,3 +221,70 @@ def test_bwd_argument_errors(fa):
     with pytest.raises(fa.FAError) as e:
         fa.fa_bwd(x, x, x, x, lse, x, 0, x, x, ws, ws.numel(), B, H, H, N, d, 0, 0.1)
     assert e.value.status == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_d64_gqa_fwd_bwd(fa, causal):
+    """Packed sequences with d = 64 and GQA (8 query heads on 2 kv heads),
+    ragged lengths including an empty one: forward and backward against the
+    oracle."""
+    lengths = [1, 200, 129, 0, 513, 64]
+    Hq, Hkv, d = 8, 2, 64
+    q, k, v, do, cu = synth.qkv_varlen_bf16(41, lengths, Hq, Hkv, d, with_dout=True)
+    dev = torch.device("cuda")
+    cu_d = torch.from_numpy(cu).to(dev)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    o, lse = fa.attention_fwd_varlen(qd, kd, vd, cu_d, max(lengths), causal=causal)
+    dq, dk, dv = fa.attention_bwd_varlen(qd, kd, vd, o, lse, dod, cu_d, max(lengths), causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    scale = 1 / math.sqrt(d)
+    O, L = oracle.attn_fwd_varlen(q, k, v, cu, causal, scale)
+    assert oracle.rel_rms(o.cpu(), O) <= 5e-3 and oracle.max_abs(o.cpu(), O) <= 2e-2
+    assert float(np.max(np.abs(lse.cpu().double().numpy() - L))) <= 1e-3
+    want = oracle.attn_bwd_varlen(q, k, v, do, cu, causal, scale)
+    _check_grads((dq, dk, dv), want, f"varlen d64 gqa causal={causal}")
+
+
+def test_mqa_fwd_bwd(fa):
+    """One kv head shared by 16 query heads (the widest GQA group): dK, dV sum
+    16 heads' contributions."""
+    (q, k, v, do), got = _fwd_bwd_padded(fa, 2, 640, 16, 1, 128, True, seed=43)
+    want = oracle.attn_bwd(q, k, v, do, True, 1 / math.sqrt(128))
+    _check_grads(got, want, "mqa")
+
+
+def test_max_sequence_length(fa):
+    """The longest sequence the varlen scheduler takes (131072 tokens, one
+    sequence beside two short ones, causal, GQA 2:1): O and LSE on 32 seeded
+    rows of each query head, dQ on the same rows, against the oracle's
+    row-sampled forward and backward (padded layout of the long sequence)."""
+    N, Hq, Hkv, d = 131072, 2, 1, 128
+    lengths = [N, 5, 300]
+    q, k, v, do, cu = synth.qkv_varlen_bf16(47, lengths, Hq, Hkv, d, with_dout=True)
+    dev = torch.device("cuda")
+    cu_d = torch.from_numpy(cu).to(dev)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    o, lse = fa.attention_fwd_varlen(qd, kd, vd, cu_d, N, causal=True)
+    dq, dk, dv = fa.attention_bwd_varlen(qd, kd, vd, o, lse, dod, cu_d, N, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    scale = 1 / math.sqrt(d)
+    rows = synth.sample_rows(5, N, Hq, R=32)
+    ql, kl, vl, dol = (t[None, :N] for t in (q, k, v, do))  # the long sequence, padded layout
+    O, L = oracle.attn_fwd_rows(ql, kl, vl, True, scale, rows)
+    wq, _, _ = oracle.attn_bwd_rows(ql, kl, vl, dol, True, scale, rows)
+    o_c, lse_c, dq_c = o.cpu(), lse.cpu(), dq.cpu()
+    for h in range(Hq):
+        got_o = o_c[rows[h], h].double().numpy()
+        assert oracle.rel_rms(got_o, O[0, h]) <= 5e-3 and oracle.max_abs(got_o, O[0, h]) <= 2e-2
+        assert float(np.max(np.abs(lse_c[h, rows[h]].double().numpy() - L[0, h]))) <= 1e-3
+        assert oracle.rel_rms(dq_c[rows[h], h].double().numpy(), wq[0, h]) <= G_REL_RMS
+    # the short sequences packed after it, in full
+    a = N
+    sl = slice(a, None)
+    cu_s = cu[1:] - a
+    Os, Ls = oracle.attn_fwd_varlen(q[sl], k[sl], v[sl], cu_s, True, scale)
+    assert oracle.rel_rms(o_c[sl], Os) <= 5e-3
+    gs = oracle.attn_bwd_varlen(q[sl], k[sl], v[sl], do[sl], cu_s, True, scale)
+    _check_grads((dq_c[sl], dk.cpu()[sl], dv.cpu()[sl]), gs, "short sequences after the longest")
