@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-bwd", action="store_true", help="time the forward pass only")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--shape", default=None,
                     help="B,Hq,Hkv,N,d,causal: another workload (profiling captures; not the headline line)")
@@ -454,37 +454,68 @@ def run_ours(args):
                     "traffic": traffic_for(dom["kernel"], step_shape(B, Hq, Hkv, N, d, causal)), "peak_source": f"{pk['source']} HBM copy",
                     "kernels": kernels}
 
-    # end to end through the public API with host buffers (pinned), copies timed
+    # end to end through the public API with host buffers (pinned), copies
+    # timed: every step copies its inputs in and its results out, on streams
+    # of their own so that step i's compute overlaps step i+1's inputs and
+    # step i-1's results (two device buffers per tensor, as a training loop
+    # that prefetches its next batch would hold)
     e2e = None
     if args.e2e_steps > 0:
         pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
-        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
-        h2d = sum(t.numel() * t.element_size() for t in (pin if with_bwd else pin[:3]))
-        d2h = sum(t.numel() * t.element_size() for t in (outs_h if with_bwd else outs_h[:2]))
+        n_in = 4 if with_bwd else 3
+        n_out = 5 if with_bwd else 2
+        dev_in = [[q, k, v, do], [torch.empty_like(t) for t in (q, k, v, do)]]
+        dev_out = [[o, lse, dq, dk, dv], [torch.empty_like(t) for t in (o, lse, dq, dk, dv)]]
+        ws_pair = [ws, torch.empty_like(ws)]
+        outs_h = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)] for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in pin[:n_in])
+        d2h = sum(t.numel() * t.element_size() for t in outs_h[0][:n_out])
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_read = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(b):
+            qq, kk, vv, dd = dev_in[b]
+            oo, ll, gq, gk, gv = dev_out[b]
+            fa.fa_fwd(qq, kk, vv, oo, ll, B, Hq, Hkv, N, d, int(causal), scale, sptr)
+            if with_bwd:
+                fa.fa_bwd(qq, kk, vv, oo, ll, dd, gq, gk, gv, ws_pair[b], ws_bytes, B, Hq, Hkv, N, d, int(causal),
+                          scale, sptr)
+
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize(dev)
         if pg:
             pg.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            q.copy_(pin[0], non_blocking=True)
-            k.copy_(pin[1], non_blocking=True)
-            v.copy_(pin[2], non_blocking=True)
-            if with_bwd:
-                do.copy_(pin[3], non_blocking=True)
-            step()
-            outs_h[0].copy_(o, non_blocking=True)
-            outs_h[1].copy_(lse, non_blocking=True)
-            if with_bwd:
-                outs_h[2].copy_(dq, non_blocking=True)
-                outs_h[3].copy_(dk, non_blocking=True)
-                outs_h[4].copy_(dv, non_blocking=True)
-        e1.record(stream)
+        e0.record(s_in)
+        for i in range(args.e2e_steps):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev_done[b])  # step i-2's compute is done with buffer b's inputs
+            with torch.cuda.stream(s_in):
+                for j in range(n_in):
+                    dev_in[b][j].copy_(pin[j], non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_read[b])  # step i-2's results in buffer b are back on the host
+            e2e_step(b)
+            ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                for j in range(n_out):
+                    outs_h[b][j].copy_(dev_out[b][j], non_blocking=True)
+            ev_read[b].record(s_out)
+        e1.record(s_out)
         torch.cuda.synchronize(dev)
+        if fa.fa_get_status(sptr) != fa.FA_OK:
+            raise SystemExit("device status error in the end-to-end pass")
         e_ms = e0.elapsed_time(e1)
         e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": f_step * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "overlap": "inputs in, compute, results out on three streams with two device buffers per tensor; "
+                          "every step copies all of its inputs in and all of its results out"}
 
     cpu = None
     if rank == 0 and world == 1:
