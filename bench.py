@@ -236,6 +236,53 @@ def max_over_ranks(pg, dev, value):
     return float(t.item())
 
 
+E2E_OVERLAP = ("inputs in, compute, results out on three streams with two device buffers per tensor; "
+               "every step copies all of its inputs in and all of its results out")
+
+
+def e2e_pipelined(torch, dev, stream, pin_in, ins0, outs0, launch, steps, pg=None):
+    """End-to-end time of `steps` steps through the public API: step i copies
+    its inputs from the pinned host tensors `pin_in` into device buffers,
+    runs launch(ins, outs, b) on `stream`, and copies `outs` back into pinned
+    host buffers. Inputs in, compute and results out run on three streams
+    with two device buffers per tensor (b = i % 2), so that a step's compute
+    overlaps the next step's inputs and the previous step's results, as a
+    training loop that prefetches its next batch would. Returns the
+    milliseconds (max over ranks) and the bytes copied each way per step."""
+    ins = [list(ins0), [torch.empty_like(t) for t in ins0]]
+    outs = [list(outs0), [torch.empty_like(t) for t in outs0]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs0] for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in, ev_done, ev_read = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    e0.record(s_in)
+    for i in range(steps):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(ev_done[b])  # step i-2's compute is done with buffer b's inputs
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(ins[b], pin_in):
+                dst.copy_(src, non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_read[b])  # step i-2's results in buffer b are back on the host
+        launch(ins[b], outs[b], b)
+        ev_done[b].record(stream)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            for dst, src in zip(host_out[b], outs[b]):
+                dst.copy_(src, non_blocking=True)
+        ev_read[b].record(s_out)
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
+    e_ms = max_over_ranks(pg, dev, e0.elapsed_time(e1))
+    return e_ms, sum(t.numel() * t.element_size() for t in pin_in), sum(t.numel() * t.element_size() for t in host_out[0])
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -454,68 +501,27 @@ def run_ours(args):
                     "traffic": traffic_for(dom["kernel"], step_shape(B, Hq, Hkv, N, d, causal)), "peak_source": f"{pk['source']} HBM copy",
                     "kernels": kernels}
 
-    # end to end through the public API with host buffers (pinned), copies
-    # timed: every step copies its inputs in and its results out, on streams
-    # of their own so that step i's compute overlaps step i+1's inputs and
-    # step i-1's results (two device buffers per tensor, as a training loop
-    # that prefetches its next batch would hold)
+    # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if args.e2e_steps > 0:
-        pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
         n_in = 4 if with_bwd else 3
         n_out = 5 if with_bwd else 2
-        dev_in = [[q, k, v, do], [torch.empty_like(t) for t in (q, k, v, do)]]
-        dev_out = [[o, lse, dq, dk, dv], [torch.empty_like(t) for t in (o, lse, dq, dk, dv)]]
+        pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)][:n_in]
         ws_pair = [ws, torch.empty_like(ws)]
-        outs_h = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)] for _ in range(2)]
-        h2d = sum(t.numel() * t.element_size() for t in pin[:n_in])
-        d2h = sum(t.numel() * t.element_size() for t in outs_h[0][:n_out])
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev_in = [torch.cuda.Event() for _ in range(2)]
-        ev_done = [torch.cuda.Event() for _ in range(2)]
-        ev_read = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step(b):
-            qq, kk, vv, dd = dev_in[b]
-            oo, ll, gq, gk, gv = dev_out[b]
-            fa.fa_fwd(qq, kk, vv, oo, ll, B, Hq, Hkv, N, d, int(causal), scale, sptr)
+        def e2e_step(ins, outs, b):
+            fa.fa_fwd(ins[0], ins[1], ins[2], outs[0], outs[1], B, Hq, Hkv, N, d, int(causal), scale, sptr)
             if with_bwd:
-                fa.fa_bwd(qq, kk, vv, oo, ll, dd, gq, gk, gv, ws_pair[b], ws_bytes, B, Hq, Hkv, N, d, int(causal),
-                          scale, sptr)
+                fa.fa_bwd(ins[0], ins[1], ins[2], outs[0], outs[1], ins[3], outs[2], outs[3], outs[4], ws_pair[b],
+                          ws_bytes, B, Hq, Hkv, N, d, int(causal), scale, sptr)
 
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(dev)
-        if pg:
-            pg.barrier()
-        e0.record(s_in)
-        for i in range(args.e2e_steps):
-            b = i & 1
-            if i >= 2:
-                s_in.wait_event(ev_done[b])  # step i-2's compute is done with buffer b's inputs
-            with torch.cuda.stream(s_in):
-                for j in range(n_in):
-                    dev_in[b][j].copy_(pin[j], non_blocking=True)
-            ev_in[b].record(s_in)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_read[b])  # step i-2's results in buffer b are back on the host
-            e2e_step(b)
-            ev_done[b].record(stream)
-            s_out.wait_event(ev_done[b])
-            with torch.cuda.stream(s_out):
-                for j in range(n_out):
-                    outs_h[b][j].copy_(dev_out[b][j], non_blocking=True)
-            ev_read[b].record(s_out)
-        e1.record(s_out)
-        torch.cuda.synchronize(dev)
+        e_ms, h2d, d2h = e2e_pipelined(torch, dev, stream, pin, [q, k, v, do][:n_in], [o, lse, dq, dk, dv][:n_out],
+                                       e2e_step, args.e2e_steps, pg)
         if fa.fa_get_status(sptr) != fa.FA_OK:
             raise SystemExit("device status error in the end-to-end pass")
-        e_ms = e0.elapsed_time(e1)
-        e_ms = max_over_ranks(pg, dev, e_ms)
         e2e = {"value": f_step * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-               "overlap": "inputs in, compute, results out on three streams with two device buffers per tensor; "
-                          "every step copies all of its inputs in and all of its results out"}
+               "overlap": E2E_OVERLAP}
 
     cpu = None
     if rank == 0 and world == 1:
@@ -1677,26 +1683,20 @@ def run_varlen(args):
     e2e = None
     if args.e2e_steps > 0:
         pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
-        outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(dev)
-        if pg:
-            pg.barrier()
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            for dst, src in zip((q, k, v, do), pin):
-                dst.copy_(src, non_blocking=True)
-            fwd()
-            bwd()
-            for dst, src in zip(outs, (o, lse, dq, dk, dv)):
-                dst.copy_(src, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1)
-        e_ms = max_over_ranks(pg, dev, e_ms)
+        ws_pair = [ws, torch.empty_like(ws)]
+
+        def e2e_step(ins, outs, b):
+            fa.fa_fwd_varlen(ins[0], ins[1], ins[2], outs[0], outs[1], cu, nseq, mx, T, H, H, d, 1, scale, sptr)
+            fa.fa_bwd_varlen(ins[0], ins[1], ins[2], outs[0], outs[1], ins[3], outs[2], outs[3], outs[4], ws_pair[b],
+                             wsb, cu, nseq, mx, T, H, H, d, 1, scale, sptr)
+
+        e_ms, h2d, d2h = e2e_pipelined(torch, dev, stream, pin, [q, k, v, do], [o, lse, dq, dk, dv], e2e_step,
+                                       args.e2e_steps, pg)
+        if fa.fa_get_status(sptr) != fa.FA_OK:
+            raise SystemExit("device status error in the end-to-end pass")
         e2e = {"value": 3.5 * f * world * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs)}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+               "overlap": E2E_OVERLAP}
     cpu = None
     if rank == 0 and world == 1:
         tf, n, el, cores = varlen_oracle_sample(args.cpu_budget_s, lengths, cu_h)
