@@ -1,0 +1,71 @@
+"""Why the fp8 backward keeps its P and dS products in 16 bits (CPU).
+
+The fp8 path quantises its inputs to e4m3 and the backward is checked on the
+dequantised values at 1e-2 relative RMS. Of the backward's products, dV = P^T dO,
+dK = dS^T Q and dQ = dS K multiply by P or dS, so an fp8 GEMM there (kind
+f8f6f4 takes no 16-bit operand) would need P and dS in e4m3 too. This module
+rounds them to e4m3 the way a kernel would (per 128 x 128 block, scaled so the
+block's largest magnitude is 448, then round-to-nearest-even through torch's
+float8_e4m3fn) and sums in fp32: the gradients then miss the fp64 ones by
+about 2.5% RMS, well past the bound, for any sequence length. The fp64 part
+is checked against the oracle's backward first.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+G_REL_RMS = 1e-2  # the backward's bound on dequantised inputs
+
+
+def _e4m3_blocks(m, bs=128):
+    out = np.empty_like(m)
+    for i in range(0, m.shape[0], bs):
+        for j in range(0, m.shape[1], bs):
+            blk = m[i:i + bs, j:j + bs]
+            s = np.abs(blk).max() / 448.0
+            s = s if s > 0 else 1.0
+            q = torch.from_numpy(np.ascontiguousarray(blk / s).astype(np.float32)).to(torch.float8_e4m3fn)
+            out[i:i + bs, j:j + bs] = q.double().numpy() * s
+    return out
+
+
+def _rel(a, b):
+    return float(np.sqrt(((a - b) ** 2).mean() / (b ** 2).mean()))
+
+
+@pytest.mark.parametrize("N,causal", [(256, False), (512, True)])
+def test_e4m3_p_and_ds_miss_the_gradient_bound(N, causal):
+    B, H, d = 1, 1, 64
+    q, k, v, do = (t.double().numpy() for t in synth.qkv_bf16(11, B, N, H, H, d, with_dout=True))
+    sc = 1 / math.sqrt(d)
+    Q, K, V, dO = q[0, :, 0], k[0, :, 0], v[0, :, 0], do[0, :, 0]
+    S = sc * Q @ K.T
+    if causal:
+        S = np.where(np.tril(np.ones((N, N), dtype=bool)), S, -np.inf)
+    P = np.exp(S - S.max(1, keepdims=True))
+    P /= P.sum(1, keepdims=True)
+    Dv = (dO * (P @ V)).sum(1, keepdims=True)
+    dS = P * (dO @ V.T - Dv)
+    dq, dk, dv = sc * dS @ K, sc * dS.T @ Q, P.T @ dO
+    # the same gradients as the oracle's backward
+    rq, rk, rv = oracle.attn_bwd(q, k, v, do, causal, sc)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv)):
+        np.testing.assert_allclose(got, ref[0, :, 0], rtol=0, atol=1e-10 * np.abs(ref).max())
+    f32 = np.float32
+    dS8, P8 = _e4m3_blocks(dS), _e4m3_blocks(P)
+    dq8 = sc * (dS8.astype(f32) @ K.astype(f32))
+    dk8 = sc * (dS8.T.astype(f32) @ Q.astype(f32))
+    dv8 = P8.T.astype(f32) @ dO.astype(f32)
+    errs = [_rel(dq8.astype(np.float64), dq), _rel(dk8.astype(np.float64), dk), _rel(dv8.astype(np.float64), dv)]
+    for e in errs:
+        assert 1.5 * G_REL_RMS < e < 5 * G_REL_RMS, errs
+    # the same products in 16 bits stay well inside the bound
+    bf = lambda x: torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    dq16 = sc * (bf(dS).astype(f32) @ K.astype(f32))
+    assert _rel(dq16.astype(np.float64), dq) < 0.5 * G_REL_RMS
