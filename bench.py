@@ -1026,7 +1026,8 @@ def run_fp8(args):
         fa.fa_fwd_fp8(codes[0], codes[1], codes[2], scl[0], scl[1], scl[2], o, lse, B, H, H, N, d, 1, scale, sptr)
 
     # the training step's backward, timed apart: dequantise Q, K (rotation
-    # undone) and V, then the bf16 backward with the fp8 forward's O and LSE
+    # undone) and V for the 16-bit products, then fa_bwd_fp8 (scores on the
+    # codes) with the fp8 forward's O and LSE
     import synth
     do = synth.qkv_bf16(rank + 200, B, N, H, H, d, with_dout=True)[3].to(dev)
     deq = [torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
@@ -1037,8 +1038,8 @@ def run_fp8(args):
     def backward():
         for i, rot in enumerate((True, True, False)):
             fa.fa_fp8_dequantize(codes[i], scl[i], deq[i], B, N, H, d, int(rot), sptr)
-        fa.fa_bwd(deq[0], deq[1], deq[2], o, lse, do, grads[0], grads[1], grads[2], ws, ws_bytes, B, H, H, N, d, 1,
-                  scale, sptr)
+        fa.fa_bwd_fp8(codes[0], codes[1], scl[0], scl[1], deq[0], deq[1], deq[2], o, lse, do, grads[0], grads[1],
+                      grads[2], ws, ws_bytes, B, H, H, N, d, 1, scale, sptr)
 
     # error against fp64 attention on the unquantised fp32 values (sampled rows)
     rows = fp8_sample_rows(N)
@@ -1149,8 +1150,9 @@ def run_fp8(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": 4 * args.steps,
             "backward": {"ms": b_ms, "tflops": 2.5 * flops / (b_ms * 1e-3) / 1e12,
-                         "note": "fa_fp8_dequantize x3 (Q, K unrotated) + fa_bwd with the fp8 forward's O and LSE, "
-                                 "timed apart, per GPU; flops 2.5x the forward's"}}
+                         "note": "fa_fp8_dequantize x3 (Q, K unrotated) + fa_bwd_fp8 (scores on the e4m3 codes, "
+                                 "the other products 16-bit) with the fp8 forward's O and LSE, timed apart, per GPU; "
+                                 "flops 2.5x the forward's"}}
     print(json.dumps(line), flush=True)
     return 0
 

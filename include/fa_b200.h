@@ -296,6 +296,31 @@ fa_status_t fa_fp8_dequantize(const void* codes, const float* scales, void* x, i
                               int unrotate, void* stream);
 
 /*
+ * The fp8 backward with its score products on the e4m3 codes (FA-3 summary,
+ * contribution 3: FP8 GEMMs), for the output of fa_fwd_fp8: as fa_bwd, except
+ * that S = Q K^T (dQ kernel) and S^T = K Q^T (dK/dV kernel) run on the codes
+ * (tcgen05 kind::f8f6f4, fp32 sums) with the block scales folded into the
+ * exponent, exactly as fa_fwd_fp8 forms its scores, so P matches the forward's
+ * LSE. The other products (dV = P^T dO, dK = dS^T Q, dQ = dS K, dP = dO V^T)
+ * stay 16-bit: P and dS rounded to e4m3 would leave about 2.5% RMS error in
+ * the gradients, past their 1e-2 bound.
+ *   q8, k8   DEVICE e4m3 codes [B,N,Hq,128], [B,N,Hkv,128], 16-byte aligned,
+ *            as given to fa_fwd_fp8 (rotated or not; S is the same either way);
+ *   q_scale, k_scale DEVICE fp32 [B,H,ceil(N/128)] block scales of those codes;
+ *   q, k, v  DEVICE bf16 values of the other products, in the original space:
+ *            fa_fp8_dequantize of the codes (Q and K with `unrotate` when the
+ *            codes were rotated);
+ *   o, lse   fa_fwd_fp8's output on these codes; dout, dq, dk, dv, workspace,
+ *            ws_bytes and the rest as fa_bwd (workspace fa_bwd_workspace_size).
+ *   d = 128 only (FA_ERR_UNSUPPORTED otherwise); null or misaligned code or
+ *   scale pointers return FA_ERR_INVALID_ARG. Deterministic; launches as fa_bwd.
+ */
+fa_status_t fa_bwd_fp8(const void* q8, const void* k8, const float* q_scale, const float* k_scale, const void* q,
+                       const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                       void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N, int d,
+                       int causal, float scale, void* stream);
+
+/*
  * Merge of attention partials over disjoint key sets (the multi-GPU variants
  * of the topic page "Flash Attention and Efficient Transformer Mechanisms";
  * used by context-parallel ring attention): partial t is exact attention of

@@ -51,6 +51,7 @@ _SIGS = {
     "fa_bwd_blocksparse": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_noalloc": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P],
     "fa_bwd_part": [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
+    "fa_bwd_fp8": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _I, _I, _I, _I, _I, _F, _P],
 }
 for _name, _args in _SIGS.items():
     getattr(_lib, _name).argtypes = _args
@@ -137,6 +138,14 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N
     _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                        _ptr(workspace), ws_bytes, B, Hq, Hkv, N, d, int(causal), float(scale), _stream(stream)),
            "fa_bwd")
+
+
+def fa_bwd_fp8(q8, k8, q_scale, k_scale, q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, B, Hq, Hkv, N, d,
+               causal, scale, stream=None):
+    _check(_lib.fa_bwd_fp8(_ptr(q8), _ptr(k8), _ptr(q_scale), _ptr(k_scale), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                           _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, B, Hq, Hkv,
+                           N, d, int(causal), float(scale), _stream(stream)),
+           "fa_bwd_fp8")
 
 
 def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, ws_bytes, B, Nq, Hq, Hkv, Ncache, d,
@@ -232,11 +241,24 @@ def attention_bwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, dout, causa
     """Gradients (dq, dk, dv) bf16 of sum(o * dout) for the fp8 forward (o, lse from
     attention_fwd_fp8 on these codes), with respect to the original-space inputs:
     the codes are dequantised (Q and K unrotated when they were quantised with the
-    rotation) and the bf16 backward runs on them with the fp8 forward's o and lse."""
+    rotation) for the 16-bit products, and fa_bwd_fp8 forms the scores on the
+    codes themselves, as the forward did."""
     q = dequantize_fp8(q8, q_scale, rotated, stream)
     k = dequantize_fp8(k8, k_scale, rotated, stream)
     v = dequantize_fp8(v8, v_scale, False, stream)
-    return attention_bwd(q, k, v, o, lse, dout, causal=causal, scale=scale, workspace=workspace, stream=stream)
+    import torch
+    _check_inputs(bf16=dict(q=q, k=k, v=v, o=o, dout=dout), f32=dict(lse=lse, q_scale=q_scale, k_scale=k_scale),
+                  bytes1=dict(q8=q8, k8=k8))
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = _default_scale(d, scale)
+    if workspace is None:
+        nb = fa_bwd_workspace_size(B * N, B, Hq, d)
+        workspace = torch.empty(nb, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    fa_bwd_fp8(q8, k8, q_scale, k_scale, q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace.numel(), B, Hq, Hkv,
+               N, d, causal, scale, stream)
+    return dq, dk, dv
 
 
 def attention_fwd_fp8_rotated(q, k, v, causal=False, scale=None, stream=None):

@@ -37,7 +37,7 @@ struct DeviceState {
   int cc = 0;
   int* status = nullptr;     // device address of g_status_word
   bool fwd_attr[3][2] = {};  // [bf16 d64, bf16 d128, fp8][block-sparse]
-  bool bwd_attr[2][2] = {{false, false}, {false, false}};  // [d == 128][block-sparse]
+  bool bwd_attr[2][3] = {};  // [d == 128][bf16 dense, block-sparse, fp8 scores]
   bool dec_attr[2] = {false, false};
   // the backward runs its dQ kernel beside the dK/dV kernel: a second stream
   // and two events, created on first use
@@ -227,19 +227,23 @@ SparsePlanLayout sparse_plan_layout(size_t base, int B, int Hq, int Hkv, int N, 
   return L;
 }
 
-template <int D, bool SPARSE = false>
+// F8: the score products S = Q K^T (dQ kernel) and S^T = K Q^T (dK/dV
+// kernel) run on the e4m3 codes q8, k8 (block scales in `a`); q, k, v are
+// then the bf16 values of the other products.
+template <int D, bool SPARSE = false, bool F8 = false>
 fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void* v, const void* dout,
-                       fa::BwdArgs a, long long units_dq, long long units_dkdv, int parts, cudaStream_t stream) {
+                       fa::BwdArgs a, long long units_dq, long long units_dkdv, int parts, cudaStream_t stream,
+                       const void* q8 = nullptr, const void* k8 = nullptr) {
   constexpr int STAGES = 4;
-  auto kdq = fa::fa_bwd_dq_kernel<D, STAGES, SPARSE>;
-  auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES, SPARSE>;
-  const int smem_dq = static_cast<int>(sizeof(fa::DqSmem<D, STAGES>)) + 1024;
-  const int smem_dkv = static_cast<int>(sizeof(fa::DkvSmem<D, STAGES>)) + 1024;
+  auto kdq = fa::fa_bwd_dq_kernel<D, STAGES, SPARSE, F8>;
+  auto kdkv = fa::fa_bwd_dkdv_kernel<D, STAGES, SPARSE, F8>;
+  const int smem_dq = static_cast<int>(sizeof(fa::DqSmem<D, STAGES, F8>)) + 1024;
+  const int smem_dkv = static_cast<int>(sizeof(fa::DkvSmem<D, STAGES, F8>)) + 1024;
   auto kpre = fa::fa_bwd_pre_kernel<D>;
   const int smem_pre = static_cast<int>(sizeof(fa::PreSmem)) + 128;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    bool& done = ds->bwd_attr[D == 128 ? 1 : 0][SPARSE ? 1 : 0];
+    bool& done = ds->bwd_attr[D == 128 ? 1 : 0][F8 ? 2 : (SPARSE ? 1 : 0)];
     if (!done) {
       if (cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq) != cudaSuccess ||
           cudaFuncSetAttribute(kdkv, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dkv) != cudaSuccess ||
@@ -255,6 +259,12 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
   if ((st = encode_rows(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hkv, D)) != FA_OK) return st;
   if ((st = encode_rows(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hkv, D)) != FA_OK) return st;
   if ((st = encode_rows(&tdo, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, a.Hq, D)) != FA_OK) return st;
+  // the e4m3 code tiles of the fp8 score products (unused otherwise)
+  CUtensorMap tq8 = tq, tk8 = tk;
+  if (F8) {
+    if ((st = encode_rows(&tq8, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a.Hq, D)) != FA_OK) return st;
+    if ((st = encode_rows(&tk8, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, a.Hkv, D)) != FA_OK) return st;
+  }
   a.timeout_ns = g_timeout_ns.load();
   a.status = ds->status;
   // D and LSE in base 2: one CTA per SM (a ring of 3 x 64 KB of O and dO
@@ -290,7 +300,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
           a, static_cast<int>(units_dkdv));
       if (cudaGetLastError() != cudaSuccess) return false;
     }
-    kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, akv);
+    kdkv<<<g1, fa::kThreadsBwd, smem_dkv, stream>>>(tq, tk, tv, tdo, tq8, tk8, akv);
     if (cudaGetLastError() != cudaSuccess) return false;
     if (SPARSE) {
       fa::fa_bwd_reduce_kernel<D><<<ds->sms, 256, 0, stream>>>(a);
@@ -310,7 +320,7 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
       fa::fa_bwd_rows_list_kernel<<<(rows + 7) / 8, 256, 0, st>>>(a, rows);
       if (cudaGetLastError() != cudaSuccess) return false;
     }
-    kdq<<<g2, fa::kThreadsBwd, smem_dq, st>>>(tq, tk, tv, tdo, aq);
+    kdq<<<g2, fa::kThreadsBwd, smem_dq, st>>>(tq, tk, tv, tdo, tq8, tk8, aq);
     return cudaGetLastError() == cudaSuccess;
   };
   if ((parts & FA_BWD_DKDV) && (parts & FA_BWD_DQ) && g1 > 0 && g2 > 0) {
@@ -345,7 +355,9 @@ fa_status_t launch_bwd(DeviceState* ds, const void* q, const void* k, const void
 fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dout, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                          const int* cu, int nseq, int N, int total_T, int Hq, int Hkv, int d, int causal,
-                         float scale, void* stream, int parts = FA_BWD_ALL, const uint8_t* block_mask = nullptr) {
+                         float scale, void* stream, int parts = FA_BWD_ALL, const uint8_t* block_mask = nullptr,
+                         const void* q8 = nullptr, const void* k8 = nullptr, const float* q_scale = nullptr,
+                         const float* k_scale = nullptr) {
   fa_status_t st = check_common(q, k, v, o, lse, Hq, Hkv, d, scale);
   if (st != FA_OK) return st;
   if (!dout || !dq || !dk || !dv || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) ||
@@ -413,6 +425,13 @@ fa_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void
     a.partials = reinterpret_cast<float*>(w + L.part_off);
     a.plan_max_items = static_cast<int>(L.max_items);
     a.plan_max_slots = static_cast<int>(L.max_slots);
+  }
+  if (q8 != nullptr) {
+    // fp8 scores: padded batches, d = 128 (as the fp8 forward)
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.nblk_s = static_cast<int>(nt);
+    return launch_bwd<128, false, true>(ds, q, k, v, dout, a, udq, ukv, parts, s, q8, k8);
   }
   if (block_mask != nullptr)
     return d == 128 ? launch_bwd<128, true>(ds, q, k, v, dout, a, udq, ukv, parts, s)
@@ -611,6 +630,20 @@ fa_status_t fa_bwd_part(int parts, const void* q, const void* k, const void* v, 
   if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
   return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
                       causal, scale, stream, parts);
+}
+
+fa_status_t fa_bwd_fp8(const void* q8, const void* k8, const float* q_scale, const float* k_scale, const void* q,
+                       const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+                       void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int Hq, int Hkv, int N, int d,
+                       int causal, float scale, void* stream) {
+  if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * N == 0) return FA_OK;
+  if (static_cast<long long>(B) * N > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  if (!q8 || !k8 || !aligned(q8, 16) || !aligned(k8, 16)) return FA_ERR_INVALID_ARG;
+  if (!q_scale || !k_scale || !aligned(q_scale, 4) || !aligned(k_scale, 4)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, B * N, Hq, Hkv, d,
+                      causal, scale, stream, FA_BWD_ALL, nullptr, q8, k8, q_scale, k_scale);
 }
 
 fa_status_t fa_bwd_blocksparse(const void* q, const void* k, const void* v, const unsigned char* block_mask,

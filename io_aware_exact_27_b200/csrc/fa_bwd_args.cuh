@@ -53,6 +53,11 @@ struct BwdArgs {
   int* rows_n;
   int* rows_base;
   int* rows_list;
+  // fp8 (the score products on e4m3 codes): block scales [B, H, nblk_s] of
+  // the Q and K codes (value = code * scale); null for bf16
+  const float* q_scale;
+  const float* k_scale;
+  int nblk_s;
 };
 
 // Workspace layout: per query head, sequence s's rows start at

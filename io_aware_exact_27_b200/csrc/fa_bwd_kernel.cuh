@@ -39,12 +39,16 @@ __device__ __forceinline__ bool bwd_block_on(const BwdArgs& a, int hq, int qb, i
   return __ldg(a.block_mask + (static_cast<size_t>(hq) * a.nqb + qb) * a.nqb + kb) != 0;
 }
 // ------------------------------------------------------------------ dQ
-template <int D, int STAGES>
+template <int D, int STAGES, bool F8 = false>
 struct DqSmem {
   static constexpr int kTileBytes = kBM * D * 2;
-  alignas(1024) uint8_t q[kTileBytes];
+  static constexpr int kTile8 = kBM * D;  // a tile of e4m3 codes
+  // bf16: Q; fp8: the Q codes (S = Q K^T on e4m3; Q itself is not needed)
+  alignas(1024) uint8_t q[F8 ? kTile8 : kTileBytes];
   alignas(1024) uint8_t dout[kTileBytes];
   alignas(1024) uint8_t kv[STAGES][kTileBytes];
+  // fp8: the K codes of the blocks whose bf16 K sits in kv[2 i]
+  alignas(1024) uint8_t k8[F8 ? STAGES / 2 : 1][F8 ? kTile8 : 1024];
   uint64_t q_full, q_empty;
   uint64_t kv_full[STAGES], kv_empty[STAGES];
   uint64_t s_full[2], dp_full, ds_ready, acc_final, acc_free;
@@ -74,12 +78,14 @@ __device__ __forceinline__ void issue_ss_nt(uint32_t d_tmem, uint32_t a_smem, ui
   issue_qk<DD>(d_tmem, a_smem, b_smem);
 }
 
-template <int D, int STAGES, bool SPARSE = false>
+template <int D, int STAGES, bool SPARSE = false, bool F8 = false>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_q8, const __grid_constant__ CUtensorMap tm_k8,
                      const BwdArgs args) {
-  using Smem = DqSmem<D, STAGES>;
+  static_assert(!(F8 && SPARSE), "fp8 backward is dense");
+  using Smem = DqSmem<D, STAGES, F8>;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -110,10 +116,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
     tmem_relinquish();
   }
   if (warp == 8 && lane == 0) {
-    prefetch_tmap(&tm_q);
+    prefetch_tmap(F8 ? &tm_q8 : &tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    if constexpr (F8) prefetch_tmap(&tm_k8);
   }
   __syncthreads();
   int num_units = args.num_units;
@@ -165,9 +172,12 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
           break;
         }
         const uint32_t qbar = smem_u32(&sm.q_full);
-        mbar_expect_tx(qbar, 2 * Smem::kTileBytes);
+        mbar_expect_tx(qbar, (F8 ? Smem::kTile8 : Smem::kTileBytes) + Smem::kTileBytes);
         const int row0 = un.tok0 + un.qb2 * kBM;
-        load_tile<D>(smem_u32(sm.q), &tm_q, qbar, un.h, row0);
+        if constexpr (F8)
+          load_tile<D, 1>(smem_u32(sm.q), &tm_q8, qbar, un.h, row0);
+        else
+          load_tile<D>(smem_u32(sm.q), &tm_q, qbar, un.h, row0);
         load_tile<D>(smem_u32(sm.dout), &tm_do, qbar, un.h, row0);
         q_issued = it + 1;
         for (int j = 0; j < nblk && ok; ++j) {
@@ -180,8 +190,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
               break;
             }
             const uint32_t bar = smem_u32(&sm.kv_full[slot]);
-            mbar_expect_tx(bar, Smem::kTileBytes);
+            // fp8: a K slot also receives the block's K codes (K slots are the even ones)
+            mbar_expect_tx(bar, Smem::kTileBytes + (F8 && kv == 0 ? Smem::kTile8 : 0));
             load_tile<D>(smem_u32(sm.kv[slot]), kv == 0 ? &tm_k : &tm_v, bar, hkv, un.tok0 + jb * kBN);
+            if constexpr (F8)
+              if (kv == 0) load_tile<D, 1>(smem_u32(sm.k8[slot / 2]), &tm_k8, bar, hkv, un.tok0 + jb * kBN);
             ++kv_prod;
           }
         }
@@ -217,7 +230,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         uint32_t slotK = kv_cons % STAGES;
         if (!(ok = wait(&sm.kv_full[slotK], (kv_cons / STAGES) & 1, 41))) break;
         ++kv_cons;
-        issue_ss_nt<D>(tS0, qa, smem_u32(sm.kv[slotK]));
+        auto issue_s = [&](uint32_t d_tmem, uint32_t slot) {
+          if constexpr (F8)
+            issue_qk<D, true>(d_tmem, qa, smem_u32(sm.k8[slot / 2]));  // e4m3 codes
+          else
+            issue_ss_nt<D>(d_tmem, qa, smem_u32(sm.kv[slot]));
+        };
+        issue_s(tS0, slotK);
         tc_commit(smem_u32(&sm.s_full[0]));
         for (int j = 0; j < nblk; ++j) {
           const uint32_t slotV = kv_cons % STAGES;
@@ -232,7 +251,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             slotKn = kv_cons % STAGES;
             if (!(ok = wait(&sm.kv_full[slotKn], (kv_cons / STAGES) & 1, 43))) break;
             ++kv_cons;
-            issue_ss_nt<D>(tS0 + ((j + 1) & 1) * 128, qa, smem_u32(sm.kv[slotKn]));
+            issue_s(tS0 + ((j + 1) & 1) * 128, slotKn);
             tc_commit(smem_u32(&sm.s_full[(j + 1) & 1]));
           }
           if (j + 1 == nblk) tc_commit(smem_u32(&sm.q_empty));  // last reads of Q and dO issued
@@ -274,9 +293,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       const float lse2 = valid ? args.lse2[wi] : INFINITY;
       const float dval = valid ? args.dvec[wi] : 0.f;
       const int limit = args.causal ? min(row, un.n - 1) : un.n - 1;
+      // fp8: the scores are in code units, scaled by the Q and K block scales
+      const float* kscale = nullptr;
+      float cq = cl;
+      if constexpr (F8) {
+        cq = cl * args.q_scale[(static_cast<size_t>(un.seq) * args.Hq + un.h) * args.nblk_s + un.qb2];
+        kscale = args.k_scale + (static_cast<size_t>(un.seq) * args.Hkv + un.h / group) * args.nblk_s;
+      }
       for (int j = 0; j < nblk; ++j) {
         const int jb = block_at(rn, rb, j);  // key block of the j-th visit
         const int sb = j & 1;
+        const float cj = F8 ? cq * kscale[jb] : cl;
         const uint32_t par = sb ? (sc1 & 1) : (sc0 & 1);
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.s_full[sb]), par, abort, args.timeout_ns));
         if (!ok) {
@@ -294,7 +321,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         const bool masked_blk = off || __any_sync(0xffffffffu, c0 + 63 > limit);
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -lse2));
+          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cj, -lse2));
           p[c] = (masked_blk && (off || c0 + c > limit)) ? 0.f : x;
         }
         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.dp_full), dpc & 1, abort, args.timeout_ns));
@@ -369,12 +396,15 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 }
 
 // ------------------------------------------------------------------ dK, dV
-template <int D, int STAGES>
+template <int D, int STAGES, bool F8 = false>
 struct DkvSmem {
   static constexpr int kTileBytes = kBM * D * 2;
-  alignas(1024) uint8_t k[kTileBytes];
+  static constexpr int kTile8 = kBM * D;  // a tile of e4m3 codes
+  alignas(1024) uint8_t k[F8 ? kTile8 : kTileBytes];  // K (fp8: its codes, for S^T only)
   alignas(1024) uint8_t v[kTileBytes];
   alignas(1024) uint8_t qo[STAGES][kTileBytes];  // Q_i, dO_i alternating
+  // fp8: the step's Q codes (S^T = K Q^T on e4m3), one per step of the ring
+  alignas(1024) uint8_t q8[F8 ? STAGES / 2 : 1][F8 ? kTile8 : 1024];
   alignas(16) float vec[STAGES / 2][2][128];     // per step: LSE2, D of the 128 query columns
   uint64_t kv_full, kv_empty;
   uint64_t qo_full[STAGES], qo_empty[STAGES];
@@ -385,13 +415,15 @@ struct DkvSmem {
   int level_count[1024];
 };
 
-template <int D, int STAGES, bool SPARSE = false>
+template <int D, int STAGES, bool SPARSE = false, bool F8 = false>
 __global__ void __launch_bounds__(kThreadsBwd, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_q8, const __grid_constant__ CUtensorMap tm_k8,
                        const BwdArgs args) {
   static_assert(STAGES % 2 == 0, "Q and dO alternate in the ring");
-  using Smem = DkvSmem<D, STAGES>;
+  static_assert(!(F8 && SPARSE), "fp8 backward is dense");
+  using Smem = DkvSmem<D, STAGES, F8>;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -423,9 +455,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
   }
   if (warp == 8 && lane == 0) {
     prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
+    prefetch_tmap(F8 ? &tm_k8 : &tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    if constexpr (F8) prefetch_tmap(&tm_q8);
   }
   __syncthreads();
   int num_units = args.num_units;
@@ -487,8 +520,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       }
       if (lane == 0) {
         const uint32_t bar = smem_u32(&sm.kv_full);
-        mbar_expect_tx(bar, 2 * Smem::kTileBytes);
-        load_tile<D>(smem_u32(sm.k), &tm_k, bar, un.h, un.tok0 + un.qb2 * kBN);
+        mbar_expect_tx(bar, (F8 ? Smem::kTile8 : Smem::kTileBytes) + Smem::kTileBytes);
+        if constexpr (F8)
+          load_tile<D, 1>(smem_u32(sm.k), &tm_k8, bar, un.h, un.tok0 + un.qb2 * kBN);
+        else
+          load_tile<D>(smem_u32(sm.k), &tm_k, bar, un.h, un.tok0 + un.qb2 * kBN);
         load_tile<D>(smem_u32(sm.v), &tm_v, bar, un.h, un.tok0 + un.qb2 * kBN);
       }
       kv_issued = it + 1;
@@ -513,9 +549,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             if (w == 0) {
               float* vec = sm.vec[(qo_prod / 2) % (STAGES / 2)][0];
               const size_t wbase = static_cast<size_t>(hq) * args.ws_stride + ws_offset(un.tok0, un.seq) + qi * kBM;
-              mbar_expect_tx(bar, 2 * Smem::kTileBytes + 1024);
+              mbar_expect_tx(bar, 2 * Smem::kTileBytes + 1024 + (F8 ? Smem::kTile8 : 0));
               bulk_load(smem_u32(vec), args.lse2 + wbase, 512, bar);
               bulk_load(smem_u32(vec + 128), args.dvec + wbase, 512, bar);
+              if constexpr (F8)
+                load_tile<D, 1>(smem_u32(sm.q8[(qo_prod / 2) % (STAGES / 2)]), &tm_q8, bar, hq, un.tok0 + qi * kBM);
             }
             load_tile<D>(smem_u32(sm.qo[slot]), w == 0 ? &tm_q : &tm_do, bar, hq, un.tok0 + qi * kBM);
           }
@@ -551,7 +589,14 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         uint32_t slotQ = qo_cons % STAGES;
         if (!(ok = wait(&sm.qo_full[slotQ], (qo_cons / STAGES) & 1, 71))) break;
         uint32_t slotO = (qo_cons + 1) % STAGES;
-        issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[slotQ]));
+        // S^T = K Q^T (fp8: on the codes; the step's Q codes sit in q8[slot / 2])
+        auto issue_st = [&](uint32_t slot) {
+          if constexpr (F8)
+            issue_qk<D, true>(tS, ka, smem_u32(sm.q8[slot / 2]));
+          else
+            issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[slot]));
+        };
+        issue_st(slotQ);
         tc_commit(smem_u32(&sm.s_full));
         issue_ss_nt<D>(tDP, va, smem_u32(sm.qo[slotO]));
         tc_commit(smem_u32(&sm.dp_full));
@@ -570,7 +615,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
             nQ = qo_cons % STAGES;
             nO = (qo_cons + 1) % STAGES;
             if (!(ok = wait(&sm.qo_full[nQ], (qo_cons / STAGES) & 1, 75))) break;
-            issue_ss_nt<D>(tS, ka, smem_u32(sm.qo[nQ]));
+            issue_st(nQ);
             tc_commit(smem_u32(&sm.s_full));
           }
           // dK += dS^T Q
@@ -618,6 +663,11 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       for (int v = 0; v < nvis; ++v, ++vstep) {
         const int st = step_of(wk, v);
         const int qi = i0 + st % nqt;
+        // fp8: the scores are in code units, scaled by the Q and K block scales
+        float cs = cl;
+        if constexpr (F8)
+          cs = cl * args.q_scale[(static_cast<size_t>(un.seq) * args.Hq + un.h * group + st / nqt) * args.nblk_s + qi] *
+               args.k_scale[(static_cast<size_t>(un.seq) * args.Hkv + un.h) * args.nblk_s + un.qb2];
         // block-sparse: the forced visit of a key tile that no query tile sees
         const bool off = SPARSE && wk.y < 0;
         const float* vec = sm.vec[vstep % (STAGES / 2)][0];
@@ -645,7 +695,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
         float p[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cl, -vec[half * 64 + c]));
+          const float x = ex2_approx(fmaf(__uint_as_float(sr[c]), cs, -vec[half * 64 + c]));
           p[c] = (masked_blk && (off || q0 + c < lo || q0 + c >= un.n)) ? 0.f : x;
         }
         {

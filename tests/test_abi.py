@@ -92,6 +92,12 @@ def test_argument_checks_before_any_device_work(lib):
     lib.fa_fwd.argtypes = [P] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float, P]
     assert lib.fa_fwd(fake, fake, fake, fake, fake, -2, 1, 1, 128, 64, 0, 0.125, None) == 1
     assert lib.fa_fwd(fake, fake, fake, fake, fake, 3, 1, 1, 0, 64, 0, 0.125, None) == 0
+    # fp8 backward: code pointers required; d = 128 only
+    lib.fa_bwd_fp8.argtypes = [P] * 14 + [ctypes.c_size_t] + [ctypes.c_int] * 6 + [ctypes.c_float, P]
+    args = [fake] * 14 + [1 << 20]
+    assert lib.fa_bwd_fp8(*([None] + args[1:]), 1, 2, 2, 256, 128, 1, 0.125, None) == 1
+    assert lib.fa_bwd_fp8(*args, 1, 2, 2, 256, 64, 1, 0.125, None) == 2
+    assert lib.fa_bwd_fp8(*args, 0, 2, 2, 256, 128, 1, 0.125, None) == 0
 
 
 def test_torch_wrappers_reject_what_the_library_cannot_read():
