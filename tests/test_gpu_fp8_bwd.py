@@ -127,3 +127,27 @@ def test_fp8_backward_argument_errors(fa):
     with pytest.raises(fa.FAError) as e:
         fa.fa_bwd_fp8(q8, k8, qs, ks, q, q, q, o, lse, do, *g, ws, nb, 1, 2, 2, 256, 64, 1, scale)
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def test_fp8_backward_gqa_matches_oracle(fa):
+    """Grouped queries (4 query heads on 2 kv heads): the per-step Q-code
+    scales of the dK/dV kernel follow the step's query head, the K-code scales
+    of the dQ kernel the query head's kv head."""
+    B, N, Hq, Hkv, d = 1, 700, 4, 2, 128
+    q, k, v, do = synth.qkv_bf16(81, B, N, Hq, Hkv, d, with_dout=True)
+    dev = torch.device("cuda")
+    q8, qs = fa.quantize_fp8(q.to(dev), rotate=True)
+    k8, ks = fa.quantize_fp8(k.to(dev), rotate=True)
+    v8, vs = fa.quantize_fp8(v.to(dev), rotate=False)
+    scale = 1 / math.sqrt(d)
+    o, lse = fa.attention_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=True, scale=scale)
+    dq, dk, dv = fa.attention_bwd_fp8(q8, k8, v8, qs, ks, vs, o, lse, do.to(dev), causal=True, scale=scale,
+                                      rotated=True)
+    torch.cuda.synchronize()
+    assert fa.fa_get_status() == fa.FA_OK
+    deq = [oracle.dequantize_f32(c.cpu().float().numpy(), sc.cpu().numpy(), unrotate=u)
+           for c, sc, u in ((q8, qs, True), (k8, ks, True), (v8, vs, False))]
+    want = oracle.attn_bwd(*deq, do, True, scale)
+    for name, g, w in zip(("dq", "dk", "dv"), (dq, dk, dv), want):
+        rr = oracle.rel_rms(g.double().cpu().numpy(), w)
+        assert rr <= G_REL_RMS, f"{name} rel-RMS {rr}"
