@@ -130,6 +130,32 @@ __device__ __forceinline__ void widen_v_tile(const uint8_t* src, uint8_t* dst, i
   }
 }
 
+// 4 x 4 transpose of 16-byte pieces over the four lanes l = 4g..4g+3: on
+// entry lane l holds pieces (row l, piece c) in p[c]; on exit it holds
+// (row 4g + c, piece l % 4) in p[c]. Two stages; in stage b a lane swaps,
+// with lane l ^ b, the pieces whose bit b differs from its own lane bit.
+__device__ __forceinline__ void transpose4_pieces(uint4 (&p)[4], int lane) {
+#pragma unroll
+  for (int b = 1; b <= 2; b <<= 1) {
+    const bool hi = lane & b;
+#pragma unroll
+    for (int c0 = 0; c0 < 4; ++c0) {
+      if (c0 & b) continue;
+      const int c1 = c0 | b;
+      const uint4 send = hi ? p[c0] : p[c1];
+      uint4 r;
+      r.x = __shfl_xor_sync(0xffffffffu, send.x, b);
+      r.y = __shfl_xor_sync(0xffffffffu, send.y, b);
+      r.z = __shfl_xor_sync(0xffffffffu, send.z, b);
+      r.w = __shfl_xor_sync(0xffffffffu, send.w, b);
+      if (hi)
+        p[c0] = r;
+      else
+        p[c1] = r;
+    }
+  }
+}
+
 __device__ __forceinline__ int num_kv_blocks(const Unit& u, int causal) {
   const int nb = (u.n + kBN - 1) / kBN;
   return causal ? min(nb, 2 * u.qb2 + 2) : nb;
@@ -644,11 +670,19 @@ __global__ void __launch_bounds__(F8 ? kThreadsFwdF8 : kThreadsFwd, 1)
 #pragma unroll
         for (int t = 0; t < 16; ++t)
           pk[t] = pack_bf16x2(__uint_as_float(orr[2 * t]) * inv_l, __uint_as_float(orr[2 * t + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+        // each lane holds four 16-byte pieces of its row; a 4 x 4 transpose
+        // over the four lanes of consecutive rows (two xor stages of
+        // shuffles) lets each store instruction write 64 contiguous bytes of
+        // each of 8 rows instead of 16 bytes of each of 32
+        uint4 pc[4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-        }
+        for (int t = 0; t < 4; ++t) pc[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        transpose4_pieces(pc, lane);
+        const int j = lane & 3;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (row - j + t < un.n)
+            *reinterpret_cast<uint4*>(orow + static_cast<ptrdiff_t>(t - j) * args.Hq * D + c + 8 * j) = pc[t];
       }
       tc_fence_before();
       __syncwarp();
